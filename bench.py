@@ -1,0 +1,428 @@
+"""Benchmark of the Forcing-KV chunk step (fkv_step) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 480p]
+                    [--impl ours|reference]
+
+Prints ONE JSON line.  Metric: chunk-steps per second per layer (a chunk step
+of one layer = score + select + compact + attend over all heads of that
+layer).  ``value`` is whole-job throughput with the inputs resident in HBM;
+``e2e`` the same metric through the same C-ABI call with the inputs copied
+from pinned host memory and the output read back inside the timed region.
+
+Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events
+on the launching stream; between timed steps the L2 is flushed by writing a
+256 MiB buffer outside the events.  The per-kernel breakdown (roofline) comes
+from a second timed pass that calls the four entry points one by one with
+events between them.  N > 1: one process per GPU (torchrun), each rank runs
+its own independent chunk step (replicas: the step has no exchange), and the
+time is the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference of this
+method) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import fkv_workloads as wl  # noqa: E402
+
+METRIC = "fkv_step chunk-steps/s per layer"
+UNIT = "chunk-steps/s per layer"
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 7700.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- work model
+
+def algorithmic(w, kept_cnt, head_role):
+    """Algorithmic FLOPs / bytes of each kernel for one step (all layers).
+
+    attention: 4 * Lq * keys * D per head (QK^T and PV), keys = kept rows + Lq;
+    scoring (frame): 2 * n_s * N * D per dynamic head (QK^T), K read once;
+    scoring (token): K candidates read once (GEMV) + q_score read once;
+    compaction: kept rows of K and V read once and written once."""
+    seg_len = w.T if w.granularity == "frame" else 1
+    rows = kept_cnt.to(torch.int64) * seg_len
+    keys = rows + w.Lq
+    elem = 2 if w.dtype == "bf16" else 4
+    attn_flops = float((4 * w.Lq * keys * w.D).sum())
+    gather_bytes = float((rows * w.D * elem * 4).sum())
+    if w.granularity == "frame":
+        n_dyn = int(head_role.sum())
+        n_s = -(-w.Lq // w.score_stride)
+        score_flops = 2.0 * n_s * w.N * w.D * n_dyn
+        score_bytes = float(n_dyn * (w.N + n_s) * w.D * elem)
+    else:
+        n_c = w.N - w.sink_tokens - w.recent_tokens
+        score_flops = 2.0 * n_c * w.D * w.L * w.H
+        score_bytes = float(w.L * w.H * (n_c + w.n_score_q) * w.D * elem)
+    return {"attn_flops": attn_flops, "gather_bytes": gather_bytes,
+            "score_flops": score_flops, "score_bytes": score_bytes}
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unavailable"], "samples": 0}
+        busy = [s for s in sm if mx is None or s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "kv_cache_compression_fkv_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel_key, workload, src_hash):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(f"{kernel_key}/{workload}")
+    if not e or e.get("source_hash") != src_hash:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def run_ours(args, rank, world, local_rank):
+    import kv_cache_compression_fkv_b200 as fkv
+    dist = None
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local_rank)
+    w = wl.get(args.workload)
+    if world > 1:  # independent problem per rank (replicas)
+        w = wl.scaled(w, seed=w.seed + 7919 * rank, layer_seeds=None if w.layer_seeds is None else
+                      tuple(s + 7919 * rank for s in w.layer_seeds))
+    x_cpu = wl.generate(w)
+    p = fkv.params_for(w)
+    stream = torch.cuda.current_stream(dev)
+    x = {k: v.to(dev) for k, v in x_cpu.items()}
+    outs = fkv.allocate(p, dev)
+    io = fkv.make_step_io(p, x, outs)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # warm-up
+    for _ in range(args.warmup):
+        fkv.step(p, x, outs, io=io)
+    torch.cuda.synchronize(dev)
+    st, det = fkv.read_status(outs["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status {st} on head {det}")
+
+    # ---- timed: fused fkv_step, inputs resident
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    with ClockSampler(local_rank) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            fkv.step(p, x, outs, io=io)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = max_over_ranks(sum(step_ms))
+    clocks = clk.summary()
+
+    # ---- per-kernel breakdown: the same kernels through the four entry points
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e = kev[i]
+        e[0].record(stream)
+        fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
+                           outs["seg_score"], outs["ws"])
+        e[1].record(stream)
+        fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
+                        x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])
+        e[2].record(stream)
+        fkv.compact_gather(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
+                           outs["k_comp"], outs["v_comp"], outs["ws"])
+        e[3].record(stream)
+        fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"], outs["v_comp"],
+                              outs["kept_cnt"], outs["out"], outs["ws"])
+        e[4].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
+            for j, n in enumerate(["score", "select", "gather", "attend"])}
+
+    # ---- e2e: host buffers in, result out, through the same call
+    pinned = {k: v.pin_memory() for k, v in x_cpu.items()}
+    out_host = {k: torch.empty(outs[k].shape, dtype=outs[k].dtype, pin_memory=True)
+                for k in ("out", "kept_idx", "kept_cnt")}
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+    e2e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+    barrier()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e2e_evs[i][0].record(stream)
+        for k, v in pinned.items():
+            x[k].copy_(v, non_blocking=True)
+        fkv.step(p, x, outs, io=io)
+        for k, v in out_host.items():
+            v.copy_(outs[k], non_blocking=True)
+        e2e_evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_evs))
+    st, det = fkv.read_status(outs["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status {st} on head {det}")
+
+    alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
+                      else torch.ones(w.L, w.H))
+    peaks, peak_kind = load_peaks()
+    units = w.L * args.steps * world
+    value = units / (total_ms / 1e3)
+    e2e_value = units / (e2e_ms / 1e3)
+    attn_tfs = alg["attn_flops"] / (part["attend"] * 1e-3) / 1e12
+    gather_gbs = alg["gather_bytes"] / (part["gather"] * 1e-3) / 1e9
+    score_tfs = alg["score_flops"] / (part["score"] * 1e-3) / 1e12
+    score_gbs = alg["score_bytes"] / (part["score"] * 1e-3) / 1e9
+    src_hash = kernel_source_hash(_attend_sources())
+    traffic = committed_traffic("attend", w.name, src_hash)
+    roof = {"bound": "tensor", "kernel": "attend_compressed", "achieved": round(attn_tfs, 2),
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(attn_tfs / peaks["bf16_tflops"], 4),
+            "peak_kind": f"{peak_kind} burst bf16 (cuBLAS 8192^3)",
+            "traffic": traffic,
+            "algorithmic_per_launch": alg["attn_flops"], "ms_per_launch": round(part["attend"], 4)}
+    kernels = {
+        "score_segments": {"ms": round(part["score"], 4), "TFLOP/s": round(score_tfs, 2),
+                           "GB/s": round(score_gbs, 1),
+                           "frac_tensor": round(score_tfs / peaks["bf16_tflops"], 4),
+                           "frac_hbm": round(score_gbs / peaks["hbm_gbs"], 4)},
+        "select_topk": {"ms": round(part["select"], 4)},
+        "compact_gather": {"ms": round(part["gather"], 4), "GB/s": round(gather_gbs, 1),
+                           "frac_hbm": round(gather_gbs / peaks["hbm_gbs"], 4),
+                           "frac_hbm_spec": round(gather_gbs / SPEC_HBM_GBS, 4)},
+        "attend_compressed": {"ms": round(part["attend"], 4), "TFLOP/s": round(attn_tfs, 2),
+                              "frac_tensor": round(attn_tfs / peaks["bf16_tflops"], 4),
+                              "frac_tensor_spec": round(attn_tfs / SPEC_BF16_TFLOPS, 4)},
+        "score_plus_attend_frac_tensor": round(
+            (alg["attn_flops"] + alg["score_flops"]) / ((part["attend"] + part["score"]) * 1e-3)
+            / 1e12 / peaks["bf16_tflops"], 4),
+    }
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic (seeded, Wan-shaped)",
+        "config": {"workload": w.name, "L": w.L, "H": w.H, "D": w.D, "T": w.T, "F": w.F, "Fc": w.Fc,
+                   "granularity": w.granularity, "kept_per_head": int(outs["kept_cnt"][0, 0]),
+                   "l2": "flushed between timed steps (256 MiB write outside the events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "impl": "ours",
+        "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": fkv.step_launches(p) * args.steps,
+        "roofline": roof,
+        "kernels": kernels,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return line
+
+
+def _attend_sources():
+    d = os.path.join(ROOT, "kv_cache_compression_fkv_b200", "csrc")
+    return sorted(f for f in os.listdir(d) if f.startswith(("attend", "simt", "sm100")))
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(w, x_cpu, budget_s=15.0):
+    """Times the fp64 oracle, as it stands, on a bounded sample: whole heads
+    (scoring, selection, compaction, attention over every query row) taken in
+    order until the budget is spent; value scaled to layer-steps per second."""
+    from oracle import fkv_oracle as orc
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    x = {k: v for k, v in x_cpu.items()}
+    heads_done, t0 = 0, time.perf_counter()
+    order = [(l, h) for l in range(w.L) for h in range(w.H)]
+    # alternate static / dynamic heads so the sample has the mix of the layer
+    if w.granularity == "frame":
+        role = x["head_role"]
+        dyn = [lh for lh in order if role[lh]]
+        sta = [lh for lh in order if not role[lh]]
+        order = [v for pair in zip(dyn, sta) for v in pair] + dyn[len(sta):] + sta[len(dyn):]
+    for (l, h) in order:
+        f64 = lambda k: wl.as_float64(x[k][l, h])  # noqa: E731
+        ks, _ = orc.head_keep(
+            granularity=w.granularity,
+            dynamic=w.granularity == "token" or bool(x["head_role"][l, h]),
+            mask_row=x["static_mask"][l, h].numpy(), k=int(x["k_per_head"][l, h]),
+            q_cur=f64("q_cur"), k_hist=f64("k_hist"), T=w.T, scale=w.scale,
+            score_stride=w.score_stride, q_score=f64("q_score") if "q_score" in x else None,
+            sink=w.sink_tokens, recent=w.recent_tokens)
+        seg_len = w.T if w.granularity == "frame" else 1
+        keys = np.concatenate([orc.compact(f64("k_hist"), ks, seg_len), f64("k_cur")])
+        vals = np.concatenate([orc.compact(f64("v_hist"), ks, seg_len), f64("v_cur")])
+        orc.attention(f64("q_cur"), keys, vals, w.scale)
+        heads_done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    layers = heads_done / w.H
+    return {"value": round(layers / dt, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads_done} of {w.L * w.H} heads of workload {w.name} (full oracle step "
+                      f"per head, every query row), {dt:.1f} s, numpy fp64",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    w = wl.get(args.workload)
+    x_cpu = wl.generate(w)
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget / max(1, args.steps))
+        if i >= args.warmup:
+            vals.append(r)
+    value = statistics.mean(v["value"] for v in vals)
+    cb = dict(vals[-1])
+    cb["value"] = round(value, 6)
+    return {
+        "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3) if value else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, Wan-shaped)",
+        "config": {"workload": w.name, "L": w.L, "H": w.H, "D": w.D, "T": w.T, "F": w.F, "Fc": w.Fc,
+                   "granularity": w.granularity},
+        "impl": "reference", "cpu_baseline": cb,
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="480p", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+    line = run_ours(args, rank, world, local_rank)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

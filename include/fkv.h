@@ -1,0 +1,207 @@
+/*
+ * fkv.h -- C ABI of the Forcing-KV chunk step for NVIDIA B200 (sm_100a).
+ *
+ * One call of fkv_step performs, for every (layer, head) of a chunk-
+ * autoregressive video DiT, the hybrid head-wise KV-cache compression of
+ * Forcing-KV and the chunk's attention over the compressed cache:
+ *
+ *   1. static heads keep a fixed, profiled set of history frames
+ *      (Forcing-KV, ai-feeds.com/i/paper/2605.09681, "关键模块" 2:
+ *      structured static pruning, positions fixed once and extracted by mask);
+ *   2. dynamic heads score every history frame ("segment") by the attention
+ *      the current chunk's queries pay to it ("关键模块" 3: history grouped by
+ *      frame, each group scored against the current queries);
+ *   3. dynamic heads keep their top-k segments ("关键模块" 3: only the most
+ *      similar few segments are kept);
+ *   4. the kept K/V rows are compacted into a dense per-head cache
+ *      ("输出与工程收益": the pruned KV replaces the original cache);
+ *   5. the chunk's queries attend to that compressed cache followed by the
+ *      chunk's own K/V ("输出与工程收益"; "与现有产品/工作流的接口" step 2).
+ *
+ * A token-granular variant (FKV_GRAN_TOKEN) implements Deep Forcing's
+ * participative compression (bxzpzcl.cn/news/2125000, section 3.1): sink and
+ * recent tokens kept whole, candidate tokens scored by phi_j = sum_r q_r.k_j
+ * and the top C kept.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every tensor argument is a DEVICE pointer owned by the caller.  The
+ *    library never allocates, frees or synchronises the host (except
+ *    fkv_read_status, which says so).  A buffer whose size is zero for the
+ *    given params (e.g. k_comp when comp_rows == 0, seg_score when there is
+ *    nothing to score) may be NULL.
+ *  - Activations are contiguous row-major [L][H][rows][D]: bf16 (uint16
+ *    storage) when dtype == FKV_DTYPE_BF16, float when FKV_DTYPE_FP32.  They
+ *    must be 16-byte aligned.  L = num_layers, H = num_heads, D = head_dim.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    All work is enqueued asynchronously on it.
+ *  - Return value: an fkv_status_t.  Host-side checks (null pointers, sizes,
+ *    alignment, enums) run before anything is enqueued; on failure nothing is
+ *    launched.  Checks that need device data (k out of range, kept rows above
+ *    the capacity, segment ids out of range) cannot fail the call: the
+ *    kernels clamp, record the first such error in the workspace status word,
+ *    and the caller reads it with fkv_read_status.
+ *  - Calls that run on the same workspace must not overlap on the GPU.
+ */
+#ifndef FKV_H_
+#define FKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FKV_ABI_VERSION 1
+
+typedef enum fkv_status {
+  FKV_OK = 0,
+  FKV_ERR_INVALID_ARG = 1, /* null pointer, unknown enum, misaligned pointer  */
+  FKV_ERR_SHAPE = 2,       /* sizes negative, inconsistent or above limits    */
+  FKV_ERR_UNSUPPORTED = 3, /* valid request this build does not implement     */
+  FKV_ERR_CUDA = 4,        /* a CUDA runtime call or a launch failed          */
+  FKV_ERR_TIMEOUT = 5,     /* (device) a bounded wait gave up                 */
+  FKV_ERR_WORKSPACE = 6,   /* workspace null, too small or not 256-B aligned  */
+  FKV_ERR_DEVICE_ARG = 7   /* (device) k, segment id or capacity out of range */
+} fkv_status_t;
+
+typedef enum fkv_dtype { FKV_DTYPE_BF16 = 0, FKV_DTYPE_FP32 = 1 } fkv_dtype_t;
+
+/* Segment = one latent frame of T tokens (Forcing-KV), or one token (the
+ * participative variant, where every head is dynamic). */
+typedef enum fkv_granularity { FKV_GRAN_FRAME = 0, FKV_GRAN_TOKEN = 1 } fkv_granularity_t;
+
+typedef struct fkv_params {
+  int32_t num_layers;    /* L >= 1: layers batched in one call (independent)  */
+  int32_t num_heads;     /* H >= 1                                             */
+  int32_t head_dim;      /* D: 128 for bf16; 4..128, multiple of 4, for fp32   */
+  int32_t frame_tokens;  /* T >= 1: tokens per latent frame                    */
+  int32_t hist_frames;   /* F >= 0: history frames; N = F*T history tokens     */
+  int32_t chunk_frames;  /* Fc >= 1: chunk frames; Lq = Fc*T queries per head  */
+  int32_t score_stride;  /* frame mode, >= 1: scoring queries are q_cur rows
+                            0, s, 2s, ... (n_s = ceil(Lq / s) rows)            */
+  int32_t n_score_q;     /* token mode, >= 1: rows of q_score per head         */
+  int32_t sink_tokens;   /* token mode: S >= 0 first history tokens, kept      */
+  int32_t recent_tokens; /* token mode: R >= 0 last history tokens, kept;
+                            S + R <= N                                         */
+  int32_t comp_rows;     /* rows per (layer, head) of k_comp / v_comp (>= 0)   */
+  float scale;           /* softmax scale of the logits, e.g. 1/sqrt(D)        */
+  int32_t dtype;         /* fkv_dtype_t                                        */
+  int32_t granularity;   /* fkv_granularity_t                                  */
+} fkv_params_t;
+
+/* All inputs and outputs of fkv_step (device pointers, caller-owned). */
+typedef struct fkv_step_io {
+  const void* q_cur;          /* [L][H][Lq][D] chunk queries                    */
+  const void* k_cur;          /* [L][H][Lq][D] chunk keys                       */
+  const void* v_cur;          /* [L][H][Lq][D] chunk values                     */
+  const void* k_hist;         /* [L][H][N][D] history keys, frame f = rows
+                                 f*T .. f*T+T-1                                 */
+  const void* v_hist;         /* [L][H][N][D] history values                    */
+  const void* q_score;        /* token mode: [L][H][n_score_q][D]; else unused  */
+  const uint8_t* head_role;   /* frame mode: [L][H], 0 = static, 1 = dynamic;
+                                 unused (may be NULL) in token mode             */
+  const uint8_t* static_mask; /* frame mode: [L][H][F], 1 = keep frame (read
+                                 for static heads only); unused in token mode   */
+  const int32_t* k_per_head;  /* [L][H]: frame mode: frames kept by a dynamic
+                                 head (0..F); token mode: C (0..N-S-R)          */
+  float* seg_score;           /* [L][H][nseg] segment scores (fkv_num_segments) */
+  int32_t* kept_idx;          /* [L][H][max_kept] kept segment ids, ascending   */
+  int32_t* kept_cnt;          /* [L][H] number of kept segments                 */
+  void* k_comp;               /* [L][H][comp_rows][D] compressed keys           */
+  void* v_comp;               /* [L][H][comp_rows][D] compressed values         */
+  void* out;                  /* [L][H][Lq][D] attention output (q dtype)       */
+} fkv_step_io_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fkv_status_string(int32_t status);
+
+/* FKV_ABI_VERSION of the loaded library. */
+int32_t fkv_abi_version(void);
+
+/* Validates params alone (no pointers) and returns the status fkv_step would
+ * return for them. */
+int32_t fkv_check_params(const fkv_params_t* p);
+
+/* Scored segments per head: F (frame mode) or the candidate count N - S - R
+ * (token mode).  Size of the last dimension of seg_score. */
+int32_t fkv_num_segments(const fkv_params_t* p, int64_t* nseg);
+
+/* Entries per head of kept_idx: F (frame mode) or N (token mode, where the
+ * kept list holds token ids: sink, selected candidates, recent). */
+int32_t fkv_max_kept(const fkv_params_t* p, int64_t* max_kept);
+
+/* Compressed-cache rows per head needed for the worst case (every segment
+ * kept): F*T in frame mode, N in token mode.  comp_rows may be smaller when
+ * the caller knows its budgets; overflow is a device error (see above). */
+int32_t fkv_max_comp_rows(const fkv_params_t* p, int64_t* rows);
+
+/* Bytes of device workspace the entry points need for these params
+ * (status word plus the scoring scratch).  Always >= 256. */
+int32_t fkv_workspace_size(const fkv_params_t* p, size_t* bytes);
+
+/* Number of kernel launches one fkv_step call enqueues for these params. */
+int32_t fkv_step_launches(const fkv_params_t* p, int32_t* launches);
+
+/* Zeroes the workspace (status word included) on `stream`.  Call once after
+ * allocating it; entry points never clear the status word themselves. */
+int32_t fkv_workspace_init(void* ws, size_t bytes, void* stream);
+
+/* Synchronises `stream`, then copies the workspace status word to the host:
+ * *device_status = first device-side error recorded since the last init
+ * (FKV_OK if none), *detail = the (layer*H + head) it was seen on, or -1.
+ * Either output pointer may be NULL. */
+int32_t fkv_read_status(const void* ws, void* stream, int32_t* device_status, int32_t* detail);
+
+/* Step 2: segment scores.
+ * Frame mode (dynamic heads only; static rows of seg_score are written 0):
+ *   seg_score[l][h][f] = sum_i sum_{j in frame f} softmax_j(scale * q_i . k_j),
+ *   q_i = q_cur[l][h][i*score_stride], softmax over the N history keys.
+ *   q_score is unused (may be NULL).
+ * Token mode (every head): seg_score[l][h][c] = sum_r q_score[l][h][r] .
+ *   k_hist[l][h][S + c] for the candidates c = 0 .. N-S-R-1 (no scale).
+ * Scores are float32.  Uses the scoring scratch of `ws`. */
+int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void* q_score,
+                           const void* k_hist, const uint8_t* head_role, float* seg_score,
+                           void* ws, void* stream);
+
+/* Steps 1 and 3: kept segment lists.
+ * Frame mode: static heads keep the frames with static_mask == 1; dynamic
+ *   heads keep the k_per_head[l][h] frames of largest seg_score, ties to the
+ *   lower frame.  kept_idx[l][h][0..cnt) ascending, kept_cnt[l][h] = cnt.
+ * Token mode: kept = [0, S) + (S + the C best candidates, ties to the lower
+ *   index) + [N-R, N), ascending; kept_cnt = S + C + R.
+ * Entries of kept_idx past kept_cnt are left untouched.
+ * k out of range is clamped to [0, nseg] and recorded as FKV_ERR_DEVICE_ARG. */
+int32_t fkv_select_topk(const fkv_params_t* p, const float* seg_score, const uint8_t* head_role,
+                        const uint8_t* static_mask, const int32_t* k_per_head, int32_t* kept_idx,
+                        int32_t* kept_cnt, void* ws, void* stream);
+
+/* Step 4: compaction.  For each (l, h), copies the history rows of the kept
+ * segments, in kept_idx order, into rows 0 .. kept_cnt*seg_len - 1 of
+ * k_comp / v_comp (seg_len = T or 1).  Bit-exact copy.  Rows past that are
+ * left untouched.  More rows than comp_rows: the copy is clamped and
+ * FKV_ERR_DEVICE_ARG recorded. */
+int32_t fkv_compact_gather(const fkv_params_t* p, const void* k_hist, const void* v_hist,
+                           const int32_t* kept_idx, const int32_t* kept_cnt, void* k_comp,
+                           void* v_comp, void* ws, void* stream);
+
+/* Step 5: out[l][h][i] = sum_j softmax_j(scale * q_i . key_j) value_j with the
+ * keys = k_comp rows 0 .. kept_cnt*seg_len - 1 followed by the Lq rows of
+ * k_cur (no causal mask), values likewise.  float32 accumulation; the output
+ * is rounded to the activation dtype.  Compressed rows past the kept count
+ * are never used. */
+int32_t fkv_attend_compressed(const fkv_params_t* p, const void* q_cur, const void* k_cur,
+                              const void* v_cur, const void* k_comp, const void* v_comp,
+                              const int32_t* kept_cnt, void* out, void* ws, void* stream);
+
+/* Steps 1-5 in one call: score (dynamic / token heads), select, compact,
+ * attend, all enqueued on `stream` in that order. */
+int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FKV_H_ */

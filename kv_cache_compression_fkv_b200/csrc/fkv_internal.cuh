@@ -1,0 +1,86 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fkv.h"
+
+namespace fkv {
+
+// Resolved sizes of one call, derived once from fkv_params_t on the host.
+struct Dims {
+  int L, H, D, T, F, Fc;
+  int LH;            // L * H
+  int64_t N;         // history tokens per head, F * T
+  int64_t Lq;        // chunk queries per head, Fc * T
+  int stride;        // frame mode scoring stride
+  int64_t n_s;       // frame mode: scoring queries per head
+  int64_t n_score_q; // token mode: q_score rows per head
+  int64_t S, R;      // token mode sink / recent tokens
+  int64_t nseg;      // scored segments per head (F, or N - S - R)
+  int64_t max_kept;  // kept_idx entries per head (F, or N)
+  int64_t seg_len;   // rows per segment (T, or 1)
+  int64_t comp_rows; // rows per head of the compressed cache
+  float scale;
+  bool bf16;
+  bool token;
+  int elem;          // bytes per activation element
+};
+
+// Workspace layout (byte offsets from the workspace base, 256-B aligned).
+struct WsLayout {
+  size_t status;     // int32[2]: first device error, detail
+  size_t part_ml;    // frame mode: float2 [LH][F][n_s] per-frame (max, sumexp)
+  size_t row_ml;     // frame mode: float2 [LH][n_s] per-row (max, sum)
+  size_t qbar;       // token mode: float [LH][D] summed scoring queries
+  size_t total;
+};
+
+WsLayout ws_layout(const Dims& d);
+
+// Records the first device-side error of a call sequence.
+__device__ __forceinline__ void report(int32_t* status, int32_t code, int32_t detail) {
+  if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, detail);
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Order-preserving map of a float to uint32 (larger float -> larger key);
+// -0.0 is folded onto +0.0 so the two compare equal, as in IEEE comparison.
+__device__ __forceinline__ uint32_t ordered_key(float x) {
+  uint32_t b = __float_as_uint(x);
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// ---- launchers (each returns cudaGetLastError() of its launches) ----------
+cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
+                                    const uint8_t* head_role, float2* part_ml, cudaStream_t s);
+cudaError_t launch_score_frame_finalize(const Dims& d, const uint8_t* head_role,
+                                        const float2* part_ml, float2* row_ml, float* seg_score,
+                                        cudaStream_t s);
+cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
+                               float* qbar, float* seg_score, cudaStream_t s);
+cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uint8_t* head_role,
+                                const uint8_t* static_mask, const int32_t* k_per_head,
+                                int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
+                                cudaStream_t s);
+cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int32_t* k_per_head,
+                                int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
+                                cudaStream_t s);
+cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
+                          const int32_t* kept_idx, const int32_t* kept_cnt, void* k_comp,
+                          void* v_comp, int32_t* status, cudaStream_t s);
+cudaError_t launch_attend_simt(const Dims& d, const void* q_cur, const void* k_cur,
+                               const void* v_cur, const void* k_comp, const void* v_comp,
+                               const int32_t* kept_cnt, void* out, cudaStream_t s);
+
+}  // namespace fkv

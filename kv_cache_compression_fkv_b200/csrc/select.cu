@@ -1,0 +1,181 @@
+// Steps 1 and 3: kept segment lists.
+//
+// Frame mode (Forcing-KV, ai-feeds.com/i/paper/2605.09681, "关键模块" 2 and 3):
+//   static heads keep the frames of their fixed mask; dynamic heads keep the k
+//   frames of largest score.  One CTA per (layer, head), one thread per frame:
+//   each thread ranks its frame against all others under the total order
+//   (score desc, index asc) and keeps it when rank < k; kept frames are then
+//   written in ascending order through a ballot/popcount prefix sum.
+//
+// Token mode (Deep Forcing, bxzpzcl.cn/news/2125000, section 3.1 steps 1-3):
+//   sink [0, S) and recent [N-R, N) are kept whole; the candidates keep their
+//   C best tokens.  One CTA per (layer, head): a most-significant-digit radix
+//   select over order-preserving 32-bit keys (4 passes of 8 bits) finds the
+//   C-th largest key t and how many keys equal to t are taken; a stable
+//   block-wide compaction then emits the chosen ids in ascending order.
+#include "fkv_internal.cuh"
+
+namespace fkv {
+
+__global__ void select_frame_kernel(int F, const float* __restrict__ seg_score,
+                                    const uint8_t* __restrict__ head_role,
+                                    const uint8_t* __restrict__ static_mask,
+                                    const int32_t* __restrict__ k_per_head,
+                                    int32_t* __restrict__ kept_idx,
+                                    int32_t* __restrict__ kept_cnt, int32_t* status) {
+  extern __shared__ uint32_t keys[];
+  __shared__ int warp_counts[32];
+  const int lh = blockIdx.x;
+  const int f = threadIdx.x;
+  const bool dyn = head_role[lh] != 0;
+  int k = 0;
+  if (dyn) {
+    k = k_per_head[lh];
+    if (k < 0 || k > F) {
+      if (f == 0) report(status, FKV_ERR_DEVICE_ARG, lh);
+      k = k < 0 ? 0 : F;
+    }
+  }
+  uint32_t key = 0;
+  if (dyn && f < F) {
+    key = ordered_key(seg_score[int64_t(lh) * F + f]);
+    keys[f] = key;
+  }
+  __syncthreads();
+  bool keep = false;
+  if (f < F) {
+    if (dyn) {
+      int rank = 0;
+      for (int g = 0; g < F; ++g) {
+        const uint32_t kg = keys[g];
+        rank += (kg > key) || (kg == key && g < f);
+      }
+      keep = rank < k;
+    } else {
+      keep = static_mask[int64_t(lh) * F + f] != 0;
+    }
+  }
+  const unsigned ballot = __ballot_sync(0xffffffffu, keep);
+  const int lane = f & 31, warp = f >> 5;
+  if (lane == 0) warp_counts[warp] = __popc(ballot);
+  __syncthreads();
+  int base = 0;
+  for (int w = 0; w < warp; ++w) base += warp_counts[w];
+  if (keep) kept_idx[int64_t(lh) * F + base + __popc(ballot & ((1u << lane) - 1u))] = f;
+  if (f == 0) {
+    int total = 0;
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) total += warp_counts[w];
+    kept_cnt[lh] = total;
+  }
+}
+
+cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uint8_t* head_role,
+                                const uint8_t* static_mask, const int32_t* k_per_head,
+                                int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
+                                cudaStream_t s) {
+  const int threads = d.F <= 32 ? 32 : ((d.F + 31) / 32) * 32;
+  select_frame_kernel<<<d.LH, threads, sizeof(uint32_t) * (d.F > 0 ? d.F : 1), s>>>(
+      d.F, seg_score, head_role, static_mask, k_per_head, kept_idx, kept_cnt, status);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+
+// Exclusive block-wide prefix count of `flag` in thread order, plus the total.
+__device__ __forceinline__ int block_excl_count(bool flag, int* warp_tot, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned b = __ballot_sync(0xffffffffu, flag);
+  if (lane == 0) warp_tot[warp] = __popc(b);
+  __syncthreads();
+  int base = 0, tot = 0;
+  for (int w = 0; w < kSelWarps; ++w) {
+    const int c = warp_tot[w];
+    base += (w < warp) ? c : 0;
+    tot += c;
+  }
+  __syncthreads();
+  *total = tot;
+  return base + __popc(b & ((1u << lane) - 1u));
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N,
+                    const float* __restrict__ phi, const int32_t* __restrict__ k_per_head,
+                    int32_t* __restrict__ kept_idx, int32_t* __restrict__ kept_cnt,
+                    int32_t* status) {
+  __shared__ unsigned hist[256];
+  __shared__ int warp_tot[kSelWarps];
+  __shared__ uint32_t s_prefix;
+  __shared__ int64_t s_need;
+  const int lh = blockIdx.x;
+  const int tid = threadIdx.x;
+  const float* ph = phi + int64_t(lh) * n_c;
+  int32_t* out = kept_idx + int64_t(lh) * N;
+  int64_t C = k_per_head[lh];
+  if (C < 0 || C > n_c) {
+    if (tid == 0) report(status, FKV_ERR_DEVICE_ARG, lh);
+    C = C < 0 ? 0 : n_c;
+  }
+  for (int64_t i = tid; i < S; i += kSelThreads) out[i] = int32_t(i);
+  for (int64_t i = tid; i < R; i += kSelThreads) out[S + C + i] = int32_t(N - R + i);
+  if (tid == 0) kept_cnt[lh] = int32_t(S + C + R);
+  if (C == 0) return;
+
+  // Radix select of the C-th largest key, most significant byte first.
+  uint32_t prefix = 0, pmask = 0;
+  int64_t need = C;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
+    __syncthreads();
+    for (int64_t j = tid; j < n_c; j += kSelThreads) {
+      const uint32_t key = ordered_key(ph[j]);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int64_t above = 0;
+      int b = 255;
+      for (; b > 0; --b) {
+        if (above + int64_t(hist[b]) >= need) break;
+        above += hist[b];
+      }
+      s_prefix = prefix | (uint32_t(b) << shift);
+      s_need = need - above;
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    need = s_need;
+    pmask |= 255u << shift;
+    __syncthreads();
+  }
+  const uint32_t t = prefix;  // exact key of the C-th largest score
+  // Stable compaction: keys > t, then the first `need` keys == t by index.
+  int64_t base = 0, eq_seen = 0;
+  for (int64_t c0 = 0; c0 < n_c; c0 += kSelThreads) {
+    const int64_t j = c0 + tid;
+    const uint32_t key = j < n_c ? ordered_key(ph[j]) : 0u;
+    const bool gt = j < n_c && key > t;
+    const bool eq = j < n_c && key == t;
+    int eq_tot, take_tot;
+    const int eq_rank = block_excl_count(eq, warp_tot, &eq_tot);
+    const bool take = gt || (eq && eq_seen + eq_rank < need);
+    const int pos = block_excl_count(take, warp_tot, &take_tot);
+    if (take) out[S + base + pos] = int32_t(S + j);
+    base += take_tot;
+    eq_seen += eq_tot;
+  }
+}
+
+cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int32_t* k_per_head,
+                                int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
+                                cudaStream_t s) {
+  select_token_kernel<<<d.LH, kSelThreads, 0, s>>>(d.nseg, d.S, d.R, d.N, seg_score, k_per_head,
+                                                   kept_idx, kept_cnt, status);
+  return cudaGetLastError();
+}
+
+}  // namespace fkv

@@ -1,0 +1,379 @@
+// CUDA-core (SIMT) kernels: fp32 path of segment scoring and of attention,
+// the finalisation of the segment mass, and the token-variant scoring.
+//
+// Frame-mode segment mass (Forcing-KV, ai-feeds.com/i/paper/2605.09681,
+// "关键模块" 3), computed in one pass over the history keys:
+//   a CTA owns (layer, head, frame f, 32 scoring queries) and produces, per
+//   query row i, the frame-local max m_{f,i} and sum l_{f,i} = sum_{j in f}
+//   2^(z_ij - m_{f,i}) of the base-2 logits z = scale*log2(e)*q.k;
+//   finalisation merges the frames of a row, M_i = max_f m_{f,i},
+//   L_i = sum_f l_{f,i} 2^(m_{f,i} - M_i), and sums
+//   mass_f = sum_i l_{f,i} 2^(m_{f,i} - M_i) / L_i over the rows in a fixed
+//   order (deterministic, no atomics).
+//
+// Attention (the chunk over the compressed cache followed by its own keys):
+//   a CTA owns 32 query rows of one (layer, head) and streams 32-key tiles of
+//   the two key ranges through shared memory with an online softmax.
+#include "fkv_internal.cuh"
+
+namespace fkv {
+
+constexpr int kBQ = 32;        // query rows per CTA
+constexpr int kBK = 32;        // keys per shared-memory tile
+constexpr int kThreads = 256;  // 8 threads per query row
+constexpr int kDMax = 128;
+constexpr int kLd = kDMax + 1; // padded row pitch (floats)
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+// Copies rows [0, n) of a [rows][D] tile (source row r at src + r*row_stride
+// elements) into shared memory as float, zero-filling rows n .. nrows-1.
+template <typename T>
+__device__ __forceinline__ void load_tile(float* dst, int nrows, const T* src, int64_t row_stride,
+                                          int n, int D) {
+  const int q4 = D / 4;
+  for (int idx = threadIdx.x; idx < nrows * q4; idx += kThreads) {
+    const int r = idx / q4, c = (idx - r * q4) * 4;
+    float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+    if (r < n) {
+      const T* p = src + int64_t(r) * row_stride + c;
+      if constexpr (sizeof(T) == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+        x0 = __low2float(a); x1 = __high2float(a); x2 = __low2float(b); x3 = __high2float(b);
+      }
+    }
+    float* q = dst + r * kLd + c;
+    q[0] = x0; q[1] = x1; q[2] = x2; q[3] = x3;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Segment mass, partial pass.  grid = (ceil(n_s / 32), F, L*H).
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t n_s, float sl2,
+                           const T* __restrict__ q_cur, const T* __restrict__ k_hist,
+                           const uint8_t* __restrict__ head_role, float2* __restrict__ part_ml) {
+  const int lh = blockIdx.z;
+  if (!head_role[lh]) return;
+  extern __shared__ float smem[];
+  float* Qs = smem;
+  float* Ks = Qs + kBQ * kLd;
+  const int f = blockIdx.y;
+  const int64_t row0 = int64_t(blockIdx.x) * kBQ;
+  const int nq = int(min64(kBQ, n_s - row0));
+  load_tile(Qs, kBQ, q_cur + (int64_t(lh) * Lq + row0 * stride) * D, int64_t(stride) * D, nq, D);
+  const int r = threadIdx.x >> 3, c8 = threadIdx.x & 7;
+  float m = -INFINITY, l = 0.f;
+  const T* kf = k_hist + (int64_t(lh) * F * T_ + int64_t(f) * T_) * D;
+  for (int k0 = 0; k0 < T_; k0 += kBK) {
+    const int nk = min(kBK, T_ - k0);
+    __syncthreads();
+    load_tile(Ks, kBK, kf + int64_t(k0) * D, D, nk, D);
+    __syncthreads();
+    float s[kBK / 8];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < kBK / 8; ++v) {
+      const int j = c8 + 8 * v;
+      float acc = 0.f;
+      for (int d = 0; d < D; ++d) acc = fmaf(Qs[r * kLd + d], Ks[j * kLd + d], acc);
+      s[v] = j < nk ? acc * sl2 : -INFINITY;
+      tmax = fmaxf(tmax, s[v]);
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, o));
+    const float mn = fmaxf(m, tmax);
+    float ps = 0.f;
+#pragma unroll
+    for (int v = 0; v < kBK / 8; ++v) ps += exp2f(s[v] - mn);
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+    l = l * exp2f(m - mn) + ps;
+    m = mn;
+  }
+  if (c8 == 0 && r < nq) part_ml[(int64_t(lh) * F + f) * n_s + row0 + r] = make_float2(m, l);
+}
+
+// Per-row merge of the frame partials.  grid = (ceil(n_s / 256), L*H).
+__global__ void score_rows_kernel(int F, int64_t n_s, const uint8_t* __restrict__ head_role,
+                                  const float2* __restrict__ part_ml, float2* __restrict__ row_ml) {
+  const int lh = blockIdx.y;
+  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (!head_role[lh] || i >= n_s) return;
+  const float2* p = part_ml + int64_t(lh) * F * n_s + i;
+  float M = -INFINITY;
+  for (int f = 0; f < F; ++f) M = fmaxf(M, p[int64_t(f) * n_s].x);
+  float Ls = 0.f;
+  for (int f = 0; f < F; ++f) {
+    const float2 ml = p[int64_t(f) * n_s];
+    Ls += ml.y * exp2f(ml.x - M);
+  }
+  row_ml[int64_t(lh) * n_s + i] = make_float2(M, Ls);
+}
+
+// mass_f = sum_i l_{f,i} 2^(m_{f,i} - M_i) / L_i.  grid = (F, L*H), 256 threads.
+__global__ void score_mass_kernel(int F, int64_t n_s, const uint8_t* __restrict__ head_role,
+                                  const float2* __restrict__ part_ml,
+                                  const float2* __restrict__ row_ml, float* __restrict__ seg_score) {
+  __shared__ float red[256];
+  const int lh = blockIdx.y, f = blockIdx.x;
+  if (!head_role[lh]) {
+    if (threadIdx.x == 0) seg_score[int64_t(lh) * F + f] = 0.f;
+    return;
+  }
+  const float2* p = part_ml + (int64_t(lh) * F + f) * n_s;
+  const float2* rm = row_ml + int64_t(lh) * n_s;
+  float acc = 0.f;
+  for (int64_t i = threadIdx.x; i < n_s; i += 256) {
+    const float2 ml = p[i], MR = rm[i];
+    acc += ml.y * exp2f(ml.x - MR.x) / MR.y;
+  }
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = 128; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) seg_score[int64_t(lh) * F + f] = red[0];
+}
+
+cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
+                                    const uint8_t* head_role, float2* part_ml, cudaStream_t s) {
+  const size_t smem = sizeof(float) * 2 * kBQ * kLd;
+  dim3 grid(unsigned((d.n_s + kBQ - 1) / kBQ), unsigned(d.F), unsigned(d.LH));
+  const float sl2 = d.scale * kLog2e;
+  if (d.bf16)
+    score_frame_partial_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
+        d.D, d.T, d.F, d.Lq, d.stride, d.n_s, sl2, static_cast<const __nv_bfloat16*>(q_cur),
+        static_cast<const __nv_bfloat16*>(k_hist), head_role, part_ml);
+  else
+    score_frame_partial_kernel<float><<<grid, kThreads, smem, s>>>(
+        d.D, d.T, d.F, d.Lq, d.stride, d.n_s, sl2, static_cast<const float*>(q_cur),
+        static_cast<const float*>(k_hist), head_role, part_ml);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score_frame_finalize(const Dims& d, const uint8_t* head_role,
+                                        const float2* part_ml, float2* row_ml, float* seg_score,
+                                        cudaStream_t s) {
+  dim3 g1(unsigned((d.n_s + 255) / 256), unsigned(d.LH));
+  score_rows_kernel<<<g1, 256, 0, s>>>(d.F, d.n_s, head_role, part_ml, row_ml);
+  dim3 g2(unsigned(d.F), unsigned(d.LH));
+  score_mass_kernel<<<g2, 256, 0, s>>>(d.F, d.n_s, head_role, part_ml, row_ml, seg_score);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Token variant (Deep Forcing, bxzpzcl.cn/news/2125000, section 3.1 step 2):
+// phi_j = sum_r q_r . k_j = (sum_r q_r) . k_j.  First qbar = sum_r q_r in fp32
+// (8 row groups per dim, combined in a fixed order), then one dot product per
+// candidate row: a GEMV bound by reading the candidate keys once.
+
+template <typename T>
+__global__ void qsum_kernel(int D, int64_t n_q, const T* __restrict__ q_score,
+                            float* __restrict__ qbar) {
+  __shared__ float part[8][kDMax];
+  const int lh = blockIdx.x;
+  const int d = threadIdx.x % kDMax, g = threadIdx.x / kDMax;
+  float acc = 0.f;
+  if (d < D) {
+    const T* q = q_score + int64_t(lh) * n_q * D + d;
+    for (int64_t r = g; r < n_q; r += 8) acc += to_f32(q[r * D]);
+  }
+  part[g][d] = acc;
+  __syncthreads();
+  if (g == 0 && d < D) {
+    float tot = 0.f;
+    for (int k = 0; k < 8; ++k) tot += part[k][d];
+    qbar[int64_t(lh) * D + d] = tot;
+  }
+}
+
+// One warp per candidate row, lanes over D in 4-element groups.
+template <typename T>
+__global__ void phi_kernel(int D, int64_t N, int64_t S, int64_t n_c, const T* __restrict__ k_hist,
+                           const float* __restrict__ qbar, float* __restrict__ phi) {
+  const int lh = blockIdx.y;
+  const int lane = threadIdx.x & 31;
+  const int warps = blockDim.x >> 5;
+  const int q4 = D / 4;
+  float qb[4] = {0.f, 0.f, 0.f, 0.f};
+  if (lane < q4)
+    for (int t = 0; t < 4; ++t) qb[t] = qbar[int64_t(lh) * D + lane * 4 + t];
+  const T* kc = k_hist + (int64_t(lh) * N + S) * D;
+  for (int64_t j = int64_t(blockIdx.x) * warps + (threadIdx.x >> 5); j < n_c;
+       j += int64_t(gridDim.x) * warps) {
+    float acc = 0.f;
+    if (lane < q4) {
+      const T* p = kc + j * D + lane * 4;
+      float x[4];
+      if constexpr (sizeof(T) == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(p);
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2*>(p);
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+        x[0] = __low2float(a); x[1] = __high2float(a); x[2] = __low2float(b); x[3] = __high2float(b);
+      }
+      for (int t = 0; t < 4; ++t) acc = fmaf(qb[t], x[t], acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) phi[int64_t(lh) * n_c + j] = acc;
+  }
+}
+
+cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
+                               float* qbar, float* seg_score, cudaStream_t s) {
+  if (d.bf16)
+    qsum_kernel<__nv_bfloat16><<<d.LH, 8 * kDMax, 0, s>>>(
+        d.D, d.n_score_q, static_cast<const __nv_bfloat16*>(q_score), qbar);
+  else
+    qsum_kernel<float><<<d.LH, 8 * kDMax, 0, s>>>(d.D, d.n_score_q,
+                                                  static_cast<const float*>(q_score), qbar);
+  const int warps = 8;
+  int64_t bx = (d.nseg + warps - 1) / warps;
+  if (bx > 4096) bx = 4096;
+  dim3 grid(unsigned(bx), unsigned(d.LH));
+  if (d.bf16)
+    phi_kernel<__nv_bfloat16><<<grid, warps * 32, 0, s>>>(
+        d.D, d.N, d.S, d.nseg, static_cast<const __nv_bfloat16*>(k_hist), qbar, seg_score);
+  else
+    phi_kernel<float><<<grid, warps * 32, 0, s>>>(d.D, d.N, d.S, d.nseg,
+                                                  static_cast<const float*>(k_hist), qbar,
+                                                  seg_score);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Attention.  grid = (ceil(Lq / 32), L*H).
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+attend_simt_kernel(int D, int64_t Lq, int64_t comp_rows, int64_t seg_len, int64_t max_kept,
+                   float sl2, const T* __restrict__ q_cur, const T* __restrict__ k_cur,
+                   const T* __restrict__ v_cur, const T* __restrict__ k_comp,
+                   const T* __restrict__ v_comp, const int32_t* __restrict__ kept_cnt,
+                   T* __restrict__ out) {
+  extern __shared__ float smem[];
+  float* Qs = smem;
+  float* Ks = Qs + kBQ * kLd;
+  float* Vs = Ks + kBK * kLd;
+  float* Ps = Vs + kBK * kLd;  // [kBQ][kBK + 1]
+  const int lh = blockIdx.y;
+  const int64_t row0 = int64_t(blockIdx.x) * kBQ;
+  const int nq = int(min64(kBQ, Lq - row0));
+  int64_t cnt = kept_cnt[lh];
+  cnt = cnt < 0 ? 0 : (cnt > max_kept ? max_kept : cnt);
+  int64_t nA = cnt * seg_len;
+  if (nA > comp_rows) nA = comp_rows;
+  load_tile(Qs, kBQ, q_cur + (int64_t(lh) * Lq + row0) * D, D, nq, D);
+  const int r = threadIdx.x >> 3, c8 = threadIdx.x & 7;
+  const int nd = D / 8;  // dims per thread: c8 + 8u
+  float o[kDMax / 8];
+#pragma unroll
+  for (int u = 0; u < kDMax / 8; ++u) o[u] = 0.f;
+  float m = -INFINITY, l = 0.f;
+  const int64_t tilesA = (nA + kBK - 1) / kBK;
+  const int64_t tiles = tilesA + (Lq + kBK - 1) / kBK;
+  for (int64_t t = 0; t < tiles; ++t) {
+    const T *kp, *vp;
+    int nk;
+    if (t < tilesA) {
+      const int64_t k0 = t * kBK;
+      nk = int(min64(kBK, nA - k0));
+      kp = k_comp + (int64_t(lh) * comp_rows + k0) * D;
+      vp = v_comp + (int64_t(lh) * comp_rows + k0) * D;
+    } else {
+      const int64_t k0 = (t - tilesA) * kBK;
+      nk = int(min64(kBK, Lq - k0));
+      kp = k_cur + (int64_t(lh) * Lq + k0) * D;
+      vp = v_cur + (int64_t(lh) * Lq + k0) * D;
+    }
+    __syncthreads();
+    load_tile(Ks, kBK, kp, D, nk, D);
+    load_tile(Vs, kBK, vp, D, nk, D);
+    __syncthreads();
+    float s[kBK / 8];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int v = 0; v < kBK / 8; ++v) {
+      const int j = c8 + 8 * v;
+      float acc = 0.f;
+      for (int d = 0; d < D; ++d) acc = fmaf(Qs[r * kLd + d], Ks[j * kLd + d], acc);
+      s[v] = j < nk ? acc * sl2 : -INFINITY;
+      tmax = fmaxf(tmax, s[v]);
+    }
+#pragma unroll
+    for (int w = 1; w < 8; w <<= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, w));
+    const float mn = fmaxf(m, tmax);
+    const float corr = exp2f(m - mn);
+    float ps = 0.f;
+#pragma unroll
+    for (int v = 0; v < kBK / 8; ++v) {
+      const float p = exp2f(s[v] - mn);
+      Ps[r * (kBK + 1) + c8 + 8 * v] = p;
+      ps += p;
+    }
+#pragma unroll
+    for (int w = 1; w < 8; w <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, w);
+    l = l * corr + ps;
+    m = mn;
+    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kDMax / 8; ++u) {
+      if (u < nd) {
+        float acc = o[u] * corr;
+        for (int j = 0; j < kBK; ++j) acc = fmaf(Ps[r * (kBK + 1) + j], Vs[j * kLd + c8 + 8 * u], acc);
+        o[u] = acc;
+      }
+    }
+  }
+  if (r < nq) {
+    T* op = out + (int64_t(lh) * Lq + row0 + r) * D;
+    const float inv = 1.f / l;
+#pragma unroll
+    for (int u = 0; u < kDMax / 8; ++u)
+      if (u < nd) op[c8 + 8 * u] = from_f32<T>(o[u] * inv);
+  }
+}
+
+cudaError_t launch_attend_simt(const Dims& d, const void* q_cur, const void* k_cur,
+                               const void* v_cur, const void* k_comp, const void* v_comp,
+                               const int32_t* kept_cnt, void* out, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (kBQ * kLd + 2 * kBK * kLd + kBQ * (kBK + 1));
+  dim3 grid(unsigned((d.Lq + kBQ - 1) / kBQ), unsigned(d.LH));
+  const float sl2 = d.scale * kLog2e;
+  cudaError_t e;
+  if (d.bf16) {
+    e = cudaFuncSetAttribute(attend_simt_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attend_simt_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
+        d.D, d.Lq, d.comp_rows, d.seg_len, d.max_kept, sl2,
+        static_cast<const __nv_bfloat16*>(q_cur), static_cast<const __nv_bfloat16*>(k_cur),
+        static_cast<const __nv_bfloat16*>(v_cur), static_cast<const __nv_bfloat16*>(k_comp),
+        static_cast<const __nv_bfloat16*>(v_comp), kept_cnt, static_cast<__nv_bfloat16*>(out));
+  } else {
+    e = cudaFuncSetAttribute(attend_simt_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return e;
+    attend_simt_kernel<float><<<grid, kThreads, smem, s>>>(
+        d.D, d.Lq, d.comp_rows, d.seg_len, d.max_kept, sl2, static_cast<const float*>(q_cur),
+        static_cast<const float*>(k_cur), static_cast<const float*>(v_cur),
+        static_cast<const float*>(k_comp), static_cast<const float*>(v_comp), kept_cnt,
+        static_cast<float*>(out));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fkv

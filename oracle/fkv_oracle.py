@@ -57,6 +57,8 @@ def segment_mass(q_rows: np.ndarray, k_hist: np.ndarray, T: int, scale: float) -
     n_s = q_rows.shape[0]
     N = k_hist.shape[0]
     F = N // T
+    if F == 0:  # empty history: nothing to score
+        return np.zeros(0)
     per_row = np.empty((n_s, F), dtype=np.float64)
     for r0 in range(0, n_s, _ROW_BLOCK):
         z = scale * (q_rows[r0:r0 + _ROW_BLOCK] @ k_hist.T)

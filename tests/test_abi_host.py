@@ -1,0 +1,116 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared
+symbol, the ctypes layout matches the C structs, and host-side validation
+returns the documented status before anything is launched."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import kv_cache_compression_fkv_b200 as fkv
+from kv_cache_compression_fkv_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fkv.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(fkv_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 14
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (fkv_\w+)", out))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_struct_layout_matches_header(tmp_path, lib):
+    prog = tmp_path / "layout.c"
+    prog.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "fkv.h"\n'
+        "int main(void){printf(\"%zu %zu %zu %zu %zu\\n\", sizeof(fkv_params_t),"
+        " offsetof(fkv_params_t, scale), offsetof(fkv_params_t, granularity),"
+        " sizeof(fkv_step_io_t), offsetof(fkv_step_io_t, out)); return 0;}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
+    got = list(map(int, subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()))
+    P, S = _lib.Params, _lib.StepIO
+    assert got == [ctypes.sizeof(P), P.scale.offset, P.granularity.offset, ctypes.sizeof(S), S.out.offset]
+
+
+def test_status_strings_and_version(lib):
+    assert lib.fkv_abi_version() == 1
+    for code in range(8):
+        assert lib.fkv_status_string(code).decode().startswith("FKV_")
+    assert lib.fkv_status_string(99) == b"FKV_ERR_UNKNOWN"
+
+
+def _p(**kw):
+    base = dict(L=1, H=4, D=128, T=32, F=6, Fc=1, dtype="bf16", score_stride=1)
+    base.update(kw)
+    return fkv.make_params(**base)
+
+
+def test_param_validation(lib):
+    chk = lambda p: lib.fkv_check_params(ctypes.byref(p))
+    assert chk(_p()) == _lib.FKV_OK
+    assert chk(_p(D=64)) == _lib.FKV_ERR_UNSUPPORTED          # bf16 path is head_dim 128
+    assert chk(_p(D=64, dtype="fp32")) == _lib.FKV_OK
+    assert chk(_p(D=66, dtype="fp32")) == _lib.FKV_ERR_UNSUPPORTED
+    assert chk(_p(T=0)) == _lib.FKV_ERR_SHAPE
+    assert chk(_p(Fc=0)) == _lib.FKV_ERR_SHAPE
+    assert chk(_p(F=0)) == _lib.FKV_OK                          # empty history is allowed
+    assert chk(_p(score_stride=0)) == _lib.FKV_ERR_SHAPE
+    assert chk(_p(F=2000)) == _lib.FKV_ERR_SHAPE
+    p = _p()
+    p.dtype = 7
+    assert chk(p) == _lib.FKV_ERR_INVALID_ARG
+    p = _p()
+    p.scale = float("nan")
+    assert chk(p) == _lib.FKV_ERR_INVALID_ARG
+    tok = _p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8)
+    assert chk(tok) == _lib.FKV_OK
+    tok.sink_tokens = 180
+    assert chk(tok) == _lib.FKV_ERR_SHAPE                       # S + R > N
+    assert lib.fkv_check_params(None) == _lib.FKV_ERR_INVALID_ARG
+
+
+def test_derived_sizes(lib):
+    s = fkv.sizes(_p())
+    assert s["nseg"] == 6 and s["max_kept"] == 6 and s["max_comp_rows"] == 192
+    # status block + (max, sum) per frame and scoring row + (max, sum) per row
+    assert s["ws_bytes"] == 256 + 4 * 6 * 32 * 8 + 4 * 32 * 8
+    t = fkv.sizes(_p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8))
+    assert t["nseg"] == 192 - 80 and t["max_kept"] == 192 and t["max_comp_rows"] == 192
+
+
+def test_null_and_misaligned_pointers_fail_before_launch(lib):
+    p = _p()
+    fake = 1 << 20  # never dereferenced: validation fails first
+    assert lib.fkv_score_segments(ctypes.byref(p), fake, None, None, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_score_segments(ctypes.byref(p), fake + 8, None, fake, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_score_segments(ctypes.byref(p), fake, None, fake, fake, fake, fake + 16, None) == _lib.FKV_ERR_WORKSPACE
+    assert lib.fkv_select_topk(ctypes.byref(p), fake, None, fake, fake, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_compact_gather(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_attend_compressed(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, None, None) == _lib.FKV_ERR_WORKSPACE
+    io = _lib.StepIO()
+    assert lib.fkv_step(ctypes.byref(p), ctypes.byref(io), fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_step(ctypes.byref(p), None, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    bad = _p(T=0)
+    assert lib.fkv_step(ctypes.byref(bad), ctypes.byref(io), fake, None) == _lib.FKV_ERR_SHAPE
+    assert lib.fkv_workspace_init(fake + 8, 512, None) == _lib.FKV_ERR_WORKSPACE
+    assert lib.fkv_read_status(None, None, None, None) == _lib.FKV_ERR_WORKSPACE

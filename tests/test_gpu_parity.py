@@ -1,0 +1,99 @@
+"""Parity of the CUDA path with the fp64 oracle on every workload.
+
+Small cases are compared on every output element; the full-size workloads
+(in the launch configuration the benchmark times) on every score, kept index
+and compacted row, and on sampled attention rows the oracle computes one by
+one (always including the first and last query row, so the ragged last tile
+is covered)."""
+import numpy as np
+import pytest
+import torch
+
+import fkv_workloads as wl
+import kv_cache_compression_fkv_b200 as fkv
+from oracle import fkv_oracle as orc
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def test_tiny_fp32_full(cuda_device):
+    w = wl.get("tiny")
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    st = parity.check_step(w, x, res)
+    assert st["sel_tie"] == 0
+
+
+def test_tiny_fp32_entry_points_one_by_one(cuda_device):
+    """Each entry point alone, fed the previous step's oracle-checked output."""
+    w = wl.get("tiny")
+    x = wl.generate(w)
+    p = fkv.params_for(w)
+    d = parity.upload(x)
+    o = fkv.allocate(p)
+    fkv.score_segments(p, d["q_cur"], None, d["k_hist"], d["head_role"], o["seg_score"], o["ws"])
+    fkv.select_topk(p, o["seg_score"], d["head_role"], d["static_mask"], d["k_per_head"],
+                    o["kept_idx"], o["kept_cnt"], o["ws"])
+    fkv.compact_gather(p, d["k_hist"], d["v_hist"], o["kept_idx"], o["kept_cnt"], o["k_comp"],
+                       o["v_comp"], o["ws"])
+    fkv.attend_compressed(p, d["q_cur"], d["k_cur"], d["v_cur"], o["k_comp"], o["v_comp"],
+                          o["kept_cnt"], o["out"], o["ws"])
+    res = {k: v.cpu() for k, v in o.items() if k != "ws"}
+    res["status"] = fkv.read_status(o["ws"])
+    parity.check_step(w, x, res)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_small_multi_tile_ragged(cuda_device, dtype):
+    """Several tiles with ragged tails everywhere: T = 200, stride 3."""
+    w = wl.scaled(wl.get("480p"), name=f"small_{dtype}", H=4, T=200, F=7, Fc=2, n_static=2,
+                  static_frames=(0, 3, 6), k_dynamic=4, score_stride=3, dtype=dtype, seed=21)
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    parity.check_step(w, x, res)
+
+
+def test_small_token_variant(cuda_device):
+    w = wl.scaled(wl.get("token14b"), name="small_token", H=3, T=64, F=9, Fc=2, n_score_q=64,
+                  sink_tokens=128, recent_tokens=128, keep_tokens=200, seed=22)
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    parity.check_step(w, x, res)
+
+
+def _full(name, n_rows):
+    w = wl.get(name)
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    rows = wl.sample_rows(w.Lq, n_rows, seed=7)
+    return w, x, res, rows
+
+
+def test_480p_full_size(cuda_device):
+    w, x, res, rows = _full("480p", 48)
+    st = parity.check_step(w, x, res, rows=rows)
+    print("480p", st)
+
+
+def test_1080p_full_size(cuda_device):
+    w, x, res, rows = _full("1080p", 16)
+    st = parity.check_step(w, x, res, rows=rows)
+    print("1080p", st)
+
+
+def test_token14b_full_size(cuda_device):
+    w, x, res, rows = _full("token14b", 16)
+    heads = [(0, h) for h in range(0, 40, 3)]
+    st = parity.check_step(w, x, res, rows=rows, heads=heads)
+    print("token14b", st)
+    # every head keeps S + C + R tokens
+    assert (res["kept_cnt"] == w.sink_tokens + w.keep_tokens + w.recent_tokens).all()
+
+
+def test_480p_30_layers(cuda_device):
+    w, x, res, rows = _full("480p_30layer", 16)
+    assert (res["kept_cnt"] == 13).all()
+    heads = [(l, h) for l in (0, 11, 29) for h in range(w.H)]
+    st = parity.check_step(w, x, res, rows=rows, heads=heads)
+    print("30 layers", st)

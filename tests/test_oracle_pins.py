@@ -293,3 +293,8 @@ def test_token_step_scores_the_candidate_rows():
         kk = np.concatenate([k_hist[0, h][kept], k_cur[0, h]])
         vv = np.concatenate([v_hist[0, h][kept], v_cur[0, h]])
         np.testing.assert_allclose(res["out"][(0, h)], _sdpa(q_cur[0, h], kk, vv, 0.5), atol=1e-12)
+
+
+def test_empty_history_keeps_nothing():
+    assert orc.segment_mass(np.ones((2, 4)), np.zeros((0, 4)), 3, 0.5).shape == (0,)
+    assert orc.top_k(np.zeros(0), 0).tolist() == []

@@ -278,7 +278,7 @@ attend_simt_kernel(int D, int64_t Lq, int64_t comp_rows, int64_t seg_len, int64_
   if (nA > comp_rows) nA = comp_rows;
   load_tile(Qs, kBQ, q_cur + (int64_t(lh) * Lq + row0) * D, D, nq, D);
   const int r = threadIdx.x >> 3, c8 = threadIdx.x & 7;
-  const int nd = D / 8;  // dims per thread: c8 + 8u
+  const int nd = (D + 7) / 8;  // dims per thread: c8 + 8u < D
   float o[kDMax / 8];
 #pragma unroll
   for (int u = 0; u < kDMax / 8; ++u) o[u] = 0.f;
@@ -331,7 +331,7 @@ attend_simt_kernel(int D, int64_t Lq, int64_t comp_rows, int64_t seg_len, int64_
     __syncwarp();
 #pragma unroll
     for (int u = 0; u < kDMax / 8; ++u) {
-      if (u < nd) {
+      if (u < nd && c8 + 8 * u < D) {
         float acc = o[u] * corr;
         for (int j = 0; j < kBK; ++j) acc = fmaf(Ps[r * (kBK + 1) + j], Vs[j * kLd + c8 + 8 * u], acc);
         o[u] = acc;
@@ -343,7 +343,7 @@ attend_simt_kernel(int D, int64_t Lq, int64_t comp_rows, int64_t seg_len, int64_
     const float inv = 1.f / l;
 #pragma unroll
     for (int u = 0; u < kDMax / 8; ++u)
-      if (u < nd) op[c8 + 8 * u] = from_f32<T>(o[u] * inv);
+      if (u < nd && c8 + 8 * u < D) op[c8 + 8 * u] = from_f32<T>(o[u] * inv);
   }
 }
 

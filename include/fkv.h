@@ -166,6 +166,31 @@ int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void*
                            const void* k_hist, const uint8_t* head_role, float* seg_score,
                            void* ws, void* stream);
 
+/* fkv_score_segments without a workspace argument, for callers that cannot
+ * allocate device memory (e.g. a plugin that a host runtime hands only its
+ * input and output buffers, or a serving loop that has reserved all of HBM
+ * up front).  The pages have no counterpart of this entry point: it is a
+ * deployment convenience of this library.
+ *
+ * Same arguments, results and host-side checks as fkv_score_segments.  The
+ * scratch lives in a static 4 MiB device array inside the library (held by
+ * every GPU that loads the library until the process exits); sizes needing
+ * more (fkv_workspace_size > 4 MiB, e.g. the 30-layer 480P batch) are
+ * rejected with FKV_ERR_WORKSPACE and nothing is launched.  It calls no
+ * cudaMalloc / cudaFree.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make
+ *    that first call before any stream capture.
+ *  - Every call on a device shares the one array and leaves its contents
+ *    behind; nothing in it has to start at zero (every partial statistic is
+ *    written before it is read).  Calls that overlap on the GPU (different
+ *    streams, or threads) race on it and must be serialised by the caller.
+ *  - Device-side errors of this call are not reported (there is no workspace
+ *    status word for the caller to read). */
+int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void* q_cur, const void* q_score,
+                                   const void* k_hist, const uint8_t* head_role, float* seg_score,
+                                   void* stream);
+
 /* Steps 1 and 3: kept segment lists.
  * Frame mode: static heads keep the frames with static_mask == 1; dynamic
  *   heads keep the k_per_head[l][h] frames of largest seg_score, ties to the

@@ -29,7 +29,7 @@ from ._lib import Params, StepIO
 __all__ = [
     "FkvError", "Params", "make_params", "params_for", "sizes", "allocate", "score_segments",
     "select_topk", "compact_gather", "attend_compressed", "step", "read_status", "library",
-    "step_launches", "make_step_io",
+    "step_launches", "make_step_io", "score_segments_noalloc",
 ]
 
 
@@ -176,6 +176,21 @@ def score_segments(p: Params, q_cur, q_score, k_hist, head_role, seg_score, ws, 
         _ptr(seg_score, "seg_score", torch.float32, n["seg"]),
         _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
     _check(st, "fkv_score_segments")
+
+
+def score_segments_noalloc(p: Params, q_cur, q_score, k_hist, head_role, seg_score, stream=None):
+    """score_segments without a workspace: for callers that cannot allocate
+    device memory.  The library's own static 4 MiB device scratch is used, so
+    sizes needing more are rejected, and calls must not overlap on the GPU."""
+    n, dt = _shapes(p), _act_dtype(p)
+    token = p.granularity == _lib.FKV_GRAN_TOKEN
+    st = _lib.load().fkv_score_segments_noalloc(
+        ctypes.byref(p), _ptr(q_cur, "q_cur", dt, n["act_cur"], optional=token),
+        _ptr(q_score, "q_score", dt, n["q_score"], optional=not token),
+        _ptr(k_hist, "k_hist", dt, n["act_hist"]),
+        _ptr(head_role, "head_role", torch.uint8, n["heads"], optional=token),
+        _ptr(seg_score, "seg_score", torch.float32, n["seg"]), _stream(stream))
+    _check(st, "fkv_score_segments_noalloc")
 
 
 def select_topk(p: Params, seg_score, head_role, static_mask, k_per_head, kept_idx, kept_cnt, ws,

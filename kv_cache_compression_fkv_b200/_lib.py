@@ -61,6 +61,7 @@ SIGNATURES = {
     "fkv_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
     "fkv_read_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
     "fkv_score_segments": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "fkv_score_segments_noalloc": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "fkv_select_topk": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "fkv_compact_gather": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "fkv_attend_compressed": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),

@@ -123,7 +123,10 @@ static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, c
   if (d.F == 0) return FKV_OK;
   float2* part = reinterpret_cast<float2*>(ws_at(ws, w.part_ml));
   float2* rows = reinterpret_cast<float2*>(ws_at(ws, w.row_ml));
-  cudaError_t e = launch_score_frame_simt(d, q_cur, k_hist, head_role, part, s);
+  // bf16: tensor-core scoring; fp32: CUDA-core scoring (fp32 accuracy mode).
+  cudaError_t e = d.bf16 ? launch_score_frame_sm100(d, q_cur, k_hist, head_role, part,
+                                                    status_ptr(ws), s)
+                         : launch_score_frame_simt(d, q_cur, k_hist, head_role, part, s);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(launch_score_frame_finalize(d, head_role, part, rows, seg_score, s));
 }
@@ -148,7 +151,10 @@ static int32_t do_gather(const Dims& d, const void* k_hist, const void* v_hist,
 static int32_t do_attend(const Dims& d, const void* q_cur, const void* k_cur, const void* v_cur,
                          const void* k_comp, const void* v_comp, const int32_t* kept_cnt,
                          void* out, void* ws, cudaStream_t s) {
-  (void)ws;
+  // bf16: tensor-core attention; fp32: CUDA-core attention (fp32 accuracy mode).
+  if (d.bf16)
+    return cuda_status(launch_attend_sm100(d, q_cur, k_cur, v_cur, k_comp, v_comp, kept_cnt, out,
+                                           status_ptr(ws), s));
   return cuda_status(launch_attend_simt(d, q_cur, k_cur, v_cur, k_comp, v_comp, kept_cnt, out, s));
 }
 

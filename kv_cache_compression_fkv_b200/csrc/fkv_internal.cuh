@@ -79,6 +79,13 @@ cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int
 cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
                           const int32_t* kept_idx, const int32_t* kept_cnt, void* k_comp,
                           void* v_comp, int32_t* status, cudaStream_t s);
+cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const void* k_hist,
+                                     const uint8_t* head_role, float2* part_ml, int32_t* status,
+                                     cudaStream_t s);
+cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_cur,
+                                const void* v_cur, const void* k_comp, const void* v_comp,
+                                const int32_t* kept_cnt, void* out, int32_t* status,
+                                cudaStream_t s);
 cudaError_t launch_attend_simt(const Dims& d, const void* q_cur, const void* k_cur,
                                const void* v_cur, const void* k_comp, const void* v_comp,
                                const int32_t* kept_cnt, void* out, cudaStream_t s);

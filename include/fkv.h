@@ -86,7 +86,8 @@ typedef struct fkv_params {
   int32_t recent_tokens; /* token mode: R >= 0 last history tokens, kept;
                             S + R <= N                                         */
   int32_t comp_rows;     /* rows per (layer, head) of k_comp / v_comp (>= 0)   */
-  float scale;           /* softmax scale of the logits, e.g. 1/sqrt(D)        */
+  float scale;           /* softmax scale of the logits, finite and > 0, e.g.
+                            1/sqrt(D)                                          */
   int32_t dtype;         /* fkv_dtype_t                                        */
   int32_t granularity;   /* fkv_granularity_t                                  */
 } fkv_params_t;

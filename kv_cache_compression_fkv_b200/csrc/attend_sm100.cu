@@ -8,16 +8,20 @@
 // accumulation, bf16 out.
 //
 // One persistent CTA per SM walks (layer*head, 128-query tile) work items.
-// Warp roles (192 threads):
-//   warps 0-3  softmax: thread t owns query row t = TMEM lane t.  Reads the
-//              128x128 fp32 logits S from TMEM, keeps a running row max m and
-//              sum l, writes P = 2^(S*scale*log2e - m) as bf16 into TMEM, and
-//              rescales the fp32 O accumulator in TMEM only when m grows by
-//              more than 2^8 (lazy rescaling: P stays <= 256, exact after the
-//              final 1/l).  Epilogue: O / l -> bf16 -> global.
-//   warp 4     TMA producer: the Q tile once per work item, then K and V
+// Warp roles (320 threads):
+//   warps 0-7  softmax: query row r = 32*(w%4) + lane (= TMEM lane r) is
+//              shared by warps w and w+4, each owning 64 of the tile's 128
+//              key columns; the two exchange their partial row max through
+//              shared memory, synchronised by a 64-arrival mbarrier per pair
+//              (bounded waits, so an aborting partner cannot hang the other).  They read the fp32
+//              logits S from TMEM, keep the running row max m (and a partial
+//              row sum l each), write P = 2^(S*scale*log2e - m) as bf16 into
+//              TMEM, and rescale the fp32 O accumulator in TMEM only when m
+//              grows by more than 2^8 (lazy rescaling: P stays <= 256, exact
+//              after the final 1/l).  Epilogue: O / l -> bf16 -> global.
+//   warp 8     TMA producer: the Q tile once per work item, then K and V
 //              tiles of 128 keys into a 3-stage ring (128-byte swizzle).
-//   warp 5     MMA issuer (one thread) and TMEM owner: S = Q K^T with both
+//   warp 9     MMA issuer (one thread) and TMEM owner: S = Q K^T with both
 //              operands in shared memory, O += P V with P read from TMEM and
 //              V (MN-major) from shared memory.
 // TMEM (512 columns): S double buffer [0,256), O [256,384), P double buffer
@@ -36,7 +40,10 @@ namespace fkv {
 namespace sm100 {
 
 constexpr int kKVStages = 3;
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 320;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kColP = 384;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
@@ -56,9 +63,14 @@ struct AttnBars {
   uint64_t o_free, mma_done;
   uint32_t tmem_base;
   int abort;
+  uint64_t xbar[2][4];      // [round parity][row quarter]: 64 arrivals (warps w, w+4)
+  float xval[2][2][128];    // [round parity][column half][row] partial row max / sum
 };
 
-constexpr size_t kAttnSmem = kOffBar + sizeof(AttnBars) + 1024;
+// No alignment slack fits under the 227 KB limit: the kernel checks that the
+// dynamic shared memory base is 1024-byte aligned and reports an error if not.
+constexpr size_t kAttnSmem = kOffBar + sizeof(AttnBars);
+static_assert(kAttnSmem <= 232448, "attention shared memory above the per-CTA limit");
 
 struct AttnArgs {
   int64_t Lq, comp_rows, seg_len, max_kept;
@@ -101,13 +113,6 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kWaitCycles) return;
 }
 
-__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
-  tmem_ld32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-  tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-  tmem_ld32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-  tmem_ld32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
-  tmem_ld_wait();
-}
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -115,8 +120,12 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_vc,
                     const __grid_constant__ CUtensorMap tm_kn,
                     const __grid_constant__ CUtensorMap tm_vn, const AttnArgs a) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = align1024(smem_raw);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {  // uniform: every thread sees the same base
+    if (threadIdx.x == 0) report(a.status, FKV_ERR_UNSUPPORTED, blockIdx.x);
+    return;
+  }
+  uint8_t* sm = smem_raw;
   AttnBars* bars = reinterpret_cast<AttnBars*>(sm + kOffBar);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,16 +141,20 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], 128);
-      mbar_init(&bars->p_full[b], 128);
+      mbar_init(&bars->s_free[b], kSoftmaxThreads);
+      mbar_init(&bars->p_full[b], kSoftmaxThreads);
       mbar_init(&bars->pv_done[b], 1);
     }
-    mbar_init(&bars->o_free, 128);
+    mbar_init(&bars->o_free, kSoftmaxThreads);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&bars->xbar[0][q], 64);
+      mbar_init(&bars->xbar[1][q], 64);
+    }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
@@ -149,7 +162,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_q);
@@ -188,7 +201,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         drain_wait(&bars->v_full[i % kKVStages], (i / kKVStages) & 1);
       if (tc > 0) drain_wait(&bars->q_full, (tc - 1) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       uint32_t it = 0, tc = 0;
@@ -243,10 +256,24 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    const int row = threadIdx.x;
-    const uint32_t lane_addr = uint32_t(warp * 32) << 16;
-    uint32_t it = 0;
+    const int row = (warp & 3) * 32 + lane;
+    const int half = warp >> 2;                 // key columns [64*half, 64*half + 64)
+    const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
+    const int quarter = warp & 3;               // rows shared by warps w and w+4
+    uint32_t it = 0, xc = 0;
     bool ok = true;
+    // Exchange of one float with the partner thread of the same row: round xc
+    // uses slot xc & 1; a slot is rewritten only two rounds later, after the
+    // partner has arrived on the round in between, i.e. after it read it.
+    auto exchange = [&](float v, float* other) -> bool {
+      const uint32_t slot = xc & 1;
+      bars->xval[slot][half][row] = v;
+      mbar_arrive(&bars->xbar[slot][quarter]);
+      if (!warp_wait(&bars->xbar[slot][quarter], (xc >> 1) & 1, abort)) return false;
+      *other = bars->xval[slot][half ^ 1][row];
+      ++xc;
+      return true;
+    };
     for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
       const Tile t = decode(a, tile);
       float m = -INFINITY, l = 0.f;
@@ -254,37 +281,55 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t sb = it & 1, su = it >> 1;
         const bool inA = j < t.nbA;
         const int64_t r0 = int64_t(inA ? j : j - t.nbA) * 128;
-        const int64_t avail = (inA ? t.nA : a.Lq) - r0;
-        const int nv = avail < 128 ? int(avail) : 128;
+        const int64_t rows_left = (inA ? t.nA : a.Lq) - r0;
+        const int nv_tile = rows_left < 128 ? int(rows_left) : 128;  // valid keys of the tile
+        const int nv = nv_tile - 64 * half < 0 ? 0 : (nv_tile - 64 * half > 64 ? 64 : nv_tile - 64 * half);
         if (!(ok = warp_wait(&bars->s_full[sb], su & 1, abort))) break;
         tc_fence_after();
-        uint32_t r[128];
-        tmem_ld128(tmem + lane_addr + sb * 128, r);
+        uint32_t r[64];
+        tmem_ld32(tmem + lane_addr + sb * 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tmem + lane_addr + sb * 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&bars->s_free[sb]);
-        float x[128];
-        float mx = -INFINITY;
+        float sv[64];
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          x[i] = i < nv ? __uint_as_float(r[i]) * a.sl2 : -INFINITY;
-          mx = fmaxf(mx, x[i]);
+        for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(r[i]);
+        if (nv < 64) {  // ragged tile: columns past the valid keys never count
+#pragma unroll
+          for (int i = 0; i < 64; ++i)
+            if (i >= nv) sv[i] = -INFINITY;
         }
-        const float m_new = fmaxf(m, mx);
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(sv[k], sv[k + 8]);
+#pragma unroll
+        for (int i = 16; i < 64; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], sv[i + k], sv[i + k + 8]);
+        float pmax = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                           fmaxf(mx8[6], mx8[7]));
+        float omax;
+        if (!(ok = exchange(pmax, &omax))) break;
+        pmax = fmaxf(pmax, omax);
+        const float m_new = fmaxf(m, pmax * a.sl2);  // scale > 0
         if (j == 0) {
           m = m_new;
         } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
-          // O holds blocks < j: wait for the last PV, then rescale it in TMEM.
+          // O holds blocks < j: wait for the last PV, then rescale this half in TMEM.
           const uint32_t pi = it - 1;
           if (!(ok = warp_wait(&bars->pv_done[pi & 1], (pi >> 1) & 1, abort))) break;
           tc_fence_after();
           const float alpha = ex2(m - m_new);
-          uint32_t o[128];
-          tmem_ld128(tmem + lane_addr + kColO, o);
 #pragma unroll
-          for (int i = 0; i < 128; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int c = 0; c < 2; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem + lane_addr + kColO + half * 64 + c * 32, o);
+            tmem_ld_wait();
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tmem_st32(tmem + lane_addr + kColO + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[c * 32]));
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem + lane_addr + kColO + half * 64 + c * 32, o);
+          }
           tmem_st_wait();
           l *= alpha;
           m = m_new;
@@ -293,32 +338,32 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const uint32_t pb = it & 1, pu = it >> 1;
         if (!(ok = warp_wait(&bars->pv_done[pb], (pu & 1) ^ 1, abort))) break;
         tc_fence_after();
-        uint32_t pk[64];
-        float sum = 0.f;
+        uint32_t pk[32];
+        float2 sum4[4];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2(x[2 * i] - m), p1 = ex2(x[2 * i + 1] - m);
-          sum += p0 + p1;
-          pk[i] = pack_bf16(p0, p1);
+        for (int k = 0; k < 4; ++k) sum4[k] = make_float2(0.f, 0.f);
+        const float2 sl2x2 = make_float2(a.sl2, a.sl2), negm2 = make_float2(-m, -m);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float2 e = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2x2, negm2);
+          const float2 p = make_float2(ex2(e.x), ex2(e.y));
+          sum4[i & 3] = fadd2(sum4[i & 3], p);
+          pk[i] = pack_bf16(p.x, p.y);
         }
-        l += sum;
-        tmem_st32(tmem + lane_addr + kColP + pb * 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tmem + lane_addr + kColP + pb * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        const float2 s2 = fadd2(fadd2(sum4[0], sum4[1]), fadd2(sum4[2], sum4[3]));
+        l += s2.x + s2.y;
+        tmem_st32(tmem + lane_addr + kColP + pb * 64 + half * 32, pk);
         tmem_st_wait();
-        if (nv < 128) {
+        if (nv_tile < 128) {
           // V rows past the valid keys may hold anything (P is 0 there, but
           // 0 * NaN is not 0): zero them before the PV MMA reads the stage.
           const uint32_t s = it % kKVStages, u = it / kKVStages;
           if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort))) break;
-          if (row >= nv) {
-            uint4* v0 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + row * 128);
-            uint4* v1 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + kRegionBytes + row * 128);
+          if (row >= nv_tile) {
+            uint4* v = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + half * kRegionBytes + row * 128);
             const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              v0[c] = z;
-              v1[c] = z;
-            }
+            for (int c = 0; c < 8; ++c) v[c] = z;
           }
           fence_proxy_async_smem();
         }
@@ -326,20 +371,24 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(&bars->p_full[pb]);
       }
       if (!ok) break;
-      // Epilogue: O / l -> bf16 -> out.
+      // Epilogue: O / l -> bf16 -> out, each thread its 64 columns.
       const uint32_t last = it - 1;
       if (!(ok = warp_wait(&bars->pv_done[last & 1], (last >> 1) & 1, abort))) break;
       tc_fence_after();
-      uint32_t o[128];
-      tmem_ld128(tmem + lane_addr + kColO, o);
+      uint32_t o[64];
+      tmem_ld32(tmem + lane_addr + kColO + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+      tmem_ld32(tmem + lane_addr + kColO + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+      tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->o_free);
-      const float inv = 1.f / l;
+      float ol;
+      if (!(ok = exchange(l, &ol))) break;
+      const float inv = 1.f / (l + ol);
       const int64_t q = int64_t(t.qt) * 128 + row;
       if (q < a.Lq) {
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t(t.lh) * a.Lq + q) * 128);
+        uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t(t.lh) * a.Lq + q) * 128 + half * 64);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
+        for (int c = 0; c < 8; ++c) {
           uint4 v;
           v.x = pack_bf16(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
           v.y = pack_bf16(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
@@ -352,7 +401,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   }
 
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

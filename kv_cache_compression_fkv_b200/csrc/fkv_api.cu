@@ -42,8 +42,7 @@ static int32_t make_dims(const fkv_params_t* p, Dims* d) {
   if (p->num_layers < 1 || p->num_heads < 1 || p->frame_tokens < 1 || p->hist_frames < 0 ||
       p->chunk_frames < 1 || p->comp_rows < 0)
     return FKV_ERR_SHAPE;
-  if (!(p->scale == p->scale) || p->scale > 3.0e38f || p->scale < -3.0e38f)
-    return FKV_ERR_INVALID_ARG;
+  if (!(p->scale > 0.f) || p->scale > 3.0e38f) return FKV_ERR_INVALID_ARG;  // finite, > 0
   d->L = p->num_layers;
   d->H = p->num_heads;
   d->D = p->head_dim;

@@ -79,9 +79,10 @@ def test_param_validation(lib):
     p = _p()
     p.dtype = 7
     assert chk(p) == _lib.FKV_ERR_INVALID_ARG
-    p = _p()
-    p.scale = float("nan")
-    assert chk(p) == _lib.FKV_ERR_INVALID_ARG
+    for bad in (float("nan"), 0.0, -0.125, float("inf")):
+        p = _p()
+        p.scale = bad
+        assert chk(p) == _lib.FKV_ERR_INVALID_ARG
     tok = _p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8)
     assert chk(tok) == _lib.FKV_OK
     tok.sink_tokens = 180

@@ -145,6 +145,13 @@ int32_t fkv_workspace_size(const fkv_params_t* p, size_t* bytes);
 /* Number of kernel launches one fkv_step call enqueues for these params. */
 int32_t fkv_step_launches(const fkv_params_t* p, int32_t* launches);
 
+/* Diagnostic: y[i] = the FMA-pipe 2^x that the attention kernel uses for a
+ * share of its softmax exponentials (Cody-Waite range reduction and a
+ * degree-3 minimax polynomial; relative error <= 8.6e-5 for -126 <= x <= 127,
+ * -inf -> +0), so that it can be tested against the hardware exp2.  x, y:
+ * device arrays of n floats. */
+int32_t fkv_exp2_emulated(const float* x, float* y, int64_t n, void* stream);
+
 /* Zeroes the workspace (status word included) on `stream`.  Call once after
  * allocating it; entry points never clear the status word themselves. */
 int32_t fkv_workspace_init(void* ws, size_t bytes, void* stream);

@@ -7,28 +7,36 @@
 // [0, kept rows) then k_cur rows [0, Lq), no causal mask; bf16 in, fp32
 // accumulation, bf16 out.
 //
-// One persistent CTA per SM walks (layer*head, 128-query tile) work items.
-// Warp roles (320 threads):
-//   warps 0-7  softmax: query row r = 32*(w%4) + lane (= TMEM lane r) is
-//              shared by warps w and w+4, each owning 64 of the tile's 128
-//              key columns; the two exchange their partial row max through
-//              shared memory, synchronised by a 64-arrival mbarrier per pair
-//              (bounded waits, so an aborting partner cannot hang the other).  They read the fp32
-//              logits S from TMEM, keep the running row max m (and a partial
-//              row sum l each), write P = 2^(S*scale*log2e - m) as bf16 into
-//              TMEM, and rescale the fp32 O accumulator in TMEM only when m
-//              grows by more than 2^8 (lazy rescaling: P stays <= 256, exact
-//              after the final 1/l).  Epilogue: O / l -> bf16 -> global.
-//   warp 8     TMA producer: the Q tile once per work item, then K and V
-//              tiles of 128 keys into a 3-stage ring (128-byte swizzle).
-//   warp 9     MMA issuer (one thread) and TMEM owner: S = Q K^T with both
-//              operands in shared memory, O += P V with P read from TMEM and
-//              V (MN-major) from shared memory.
-// TMEM (512 columns): S double buffer [0,256), O [256,384), P double buffer
-// [384,512) (bf16 pairs).  The MMA of S_{j+1} overlaps the softmax of block j,
-// and O += P_{j-1} V_{j-1} overlaps it as well.
+// Work unit = one 128-query tile of one (layer, head); one persistent CTA per
+// SM walks the units.  Inside a unit the 128-key blocks are split between two
+// streams h = 0, 1 (first and second half of the blocks) that run
+// interleaved on the tensor core, each with its own softmax warpgroup, logit
+// tile S_h and fp32 accumulator O_h in TMEM; at the end of the unit the two
+// partial softmaxes are merged (rescaled by their row maxima).  While one
+// warpgroup computes exponentials the tensor core works on the other
+// stream's MMAs.
 //
-// Key tiles past the valid rows of a range are masked (logit -> -inf) and
+// Warp roles (384 threads; warps 10-11 only complete the control warpgroup):
+//   warps 0-3 / 4-7  softmax of stream 0 / 1: thread t owns query row t
+//              (= TMEM lane t).  Reads S_h from TMEM, keeps the running row
+//              max m (base-2 logits) and sum l, writes P = 2^(S*scale*log2e
+//              - m) as bf16 pairs into the first 64 columns of S_h, and
+//              rescales O_h in TMEM only when m grows by more than 2^8 (lazy
+//              rescaling: P stays <= 256, exact after the final merge).
+//              Three of every four exponential pairs go to the MUFU unit, one
+//              to an FMA-pipe polynomial (exp2_poly2) to balance the pipes.
+//   warp 8     TMA: lane 0 loads Q (once per unit) and the K blocks, lane 1
+//              the V blocks, into 3-stage rings in the order the MMAs use
+//              them: stream 0 block j, stream 1 block j, stream 0 block j+1...
+//   warp 9     MMA issuer (one thread) and TMEM owner.  Per step j it issues
+//              O_0 += P_0 V (block j-1), S_0 = Q K^T (block j), then the same
+//              for stream 1.  tcgen05 MMAs of one thread execute in issue
+//              order, so S_h of block j overwrites P_h only after the PV that
+//              reads it, and by the time S_h is complete the previous PV into
+//              O_h is complete too (the softmax may rescale O_h right away).
+// TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
+//
+// Key blocks past the valid rows of a range are masked (logit -> -inf) and
 // their V rows zeroed in shared memory before use, so compressed-cache rows
 // past the kept count are never read as data, whatever they hold.  Every
 // mbarrier wait is bounded; on timeout the CTA records FKV_ERR_TIMEOUT, waits
@@ -40,15 +48,27 @@ namespace fkv {
 namespace sm100 {
 
 constexpr int kKVStages = 3;
-constexpr int kAttnThreads = 320;
+constexpr int kAttnThreads = 384;        // 3 warpgroups
+// Register split (setmaxnreg): the kernel is launched with kLaunchRegs per
+// thread; the control warpgroup (TMA, MMA, two idle warps) gives registers
+// back, the two softmax warpgroups take them.  Budget check, registers per
+// CTA: 384 * 168 = 64512 at launch >= 256 * 224 + 128 * 56 = 64512 after;
+// per SM sub-partition (one warp of each warpgroup): (224+224+56) * 32 =
+// 16128 <= 16384.
+constexpr int kLaunchRegs = 168;
+constexpr int kSoftmaxRegs = 224;
+constexpr int kControlRegs = 56;
+static_assert(kAttnThreads * kLaunchRegs >= 256 * kSoftmaxRegs + 128 * kControlRegs,
+              "register split exceeds the launch allocation");
 constexpr int kSoftmaxThreads = 256;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr uint32_t kColO = 256;
-constexpr uint32_t kColP = 384;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 128, true);
 constexpr float kRescaleLog2 = 8.0f;
+
+__host__ __device__ constexpr uint32_t col_s(int h) { return 128u * uint32_t(h); }
+__host__ __device__ constexpr uint32_t col_o(int h) { return 256u + 128u * uint32_t(h); }
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTileBytes;
@@ -59,12 +79,13 @@ struct AttnBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kKVStages], k_empty[kKVStages];
   uint64_t v_full[kKVStages], v_empty[kKVStages];
-  uint64_t s_full[2], s_free[2], p_full[2], pv_done[2];
-  uint64_t o_free, mma_done;
+  uint64_t s_full[2], p_full[2];  // per stream
+  uint64_t o_ready, o_free;       // per unit: both PV chains done / both O read
+  uint64_t mma_done;
+  uint64_t x_full, x_read;        // merge exchange handshake (256 arrivals each)
   uint32_t tmem_base;
   int abort;
-  uint64_t xbar[2][4];      // [round parity][row quarter]: 64 arrivals (warps w, w+4)
-  float xval[2][2][128];    // [round parity][column half][row] partial row max / sum
+  float2 xml[2][128];             // [stream][row] (row max, row sum) for the merge
 };
 
 // No alignment slack fits under the 227 KB limit: the kernel checks that the
@@ -81,13 +102,13 @@ struct AttnArgs {
   int32_t* status;
 };
 
-struct Tile {
-  int lh, qt, nbA, nb;
+struct Unit {
+  int lh, qt, nbA, nb, nb0, nb1;
   int64_t nA;
 };
 
-__device__ __forceinline__ Tile decode(const AttnArgs& a, int tile) {
-  Tile t;
+__device__ __forceinline__ Unit decode(const AttnArgs& a, int tile) {
+  Unit t;
   t.lh = tile / a.n_qtiles;
   t.qt = tile - t.lh * a.n_qtiles;
   int64_t cnt = a.kept_cnt[t.lh];
@@ -97,8 +118,18 @@ __device__ __forceinline__ Tile decode(const AttnArgs& a, int tile) {
   t.nA = nA;
   t.nbA = int((nA + 127) / 128);
   t.nb = t.nbA + int((a.Lq + 127) / 128);
+  t.nb0 = (t.nb + 1) / 2;
+  t.nb1 = t.nb - t.nb0;
   return t;
 }
+
+// Position of (stream h, its j-th block) in the unit's load / MMA order:
+// s0 b0, s1 b0, s0 b1, s1 b1, ..., then the rest of stream 0.
+__device__ __forceinline__ int seq_pos(const Unit& t, int h, int j) {
+  return j < t.nb1 ? 2 * j + h : t.nb1 + j;
+}
+// Key block index of (stream h, j).
+__device__ __forceinline__ int block_of(const Unit& t, int h, int j) { return h ? t.nb0 + j : j; }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   const bool ok = mbar_wait(bar, parity, abort);
@@ -113,6 +144,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kWaitCycles) return;
 }
 
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -139,18 +178,15 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], kSoftmaxThreads);
-      mbar_init(&bars->p_full[b], kSoftmaxThreads);
-      mbar_init(&bars->pv_done[b], 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&bars->s_full[h], 1);
+      mbar_init(&bars->p_full[h], 128);
     }
+    mbar_init(&bars->o_ready, 1);
     mbar_init(&bars->o_free, kSoftmaxThreads);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(&bars->xbar[0][q], 64);
-      mbar_init(&bars->xbar[1][q], 64);
-    }
     mbar_init(&bars->mma_done, 1);
+    mbar_init(&bars->x_full, kSoftmaxThreads);
+    mbar_init(&bars->x_read, kSoftmaxThreads);
     bars->abort = 0;
     fence_mbar_init();
   }
@@ -161,242 +197,274 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-
+  if (warp >= 8) {
+    regs_decrease<kControlRegs>();
   if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // ------------------------------------------------------------ TMA producers
+    if (lane == 0) {  // Q and K
       prefetch_tmap(&tm_q);
       prefetch_tmap(&tm_kc);
-      prefetch_tmap(&tm_vc);
       prefetch_tmap(&tm_kn);
-      prefetch_tmap(&tm_vn);
-      uint32_t it_k = 0, it_v = 0, tc = 0;
+      uint32_t n = 0, tc = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
-        const Tile t = decode(a, tile);
+        const Unit t = decode(a, tile);
         if (!(ok = mbar_wait(&bars->q_empty, (tc & 1) ^ 1, abort))) break;
         mbar_expect_tx(&bars->q_full, kTileBytes);
         tma_load_tile(sm + kOffQ, &tm_q, &bars->q_full, t.qt * 128, t.lh);
         ++tc;
-        for (int j = 0; j < t.nb; ++j) {
-          const bool inA = j < t.nbA;
-          const int row = (inA ? j : j - t.nbA) * 128;
-          const uint32_t s = it_k % kKVStages, u = it_k / kKVStages;
-          if (!(ok = mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort))) break;
-          mbar_expect_tx(&bars->k_full[s], kTileBytes);
-          tma_load_tile(sm + kOffK + s * kTileBytes, inA ? &tm_kc : &tm_kn, &bars->k_full[s], row,
-                        t.lh);
-          ++it_k;
-          if (!(ok = mbar_wait(&bars->v_empty[s], (u & 1) ^ 1, abort))) break;
-          mbar_expect_tx(&bars->v_full[s], kTileBytes);
-          tma_load_tile(sm + kOffV + s * kTileBytes, inA ? &tm_vc : &tm_vn, &bars->v_full[s], row,
-                        t.lh);
-          ++it_v;
+        for (int j = 0; ok && j < t.nb0; ++j) {
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && j >= t.nb1) break;
+            const int b = block_of(t, h, j);
+            const bool inA = b < t.nbA;
+            const int row = (inA ? b : b - t.nbA) * 128;
+            const uint32_t s = n % kKVStages, u = n / kKVStages;
+            if (!(ok = mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort))) break;
+            mbar_expect_tx(&bars->k_full[s], kTileBytes);
+            tma_load_tile(sm + kOffK + s * kTileBytes, inA ? &tm_kc : &tm_kn, &bars->k_full[s],
+                          row, t.lh);
+            ++n;
+          }
         }
       }
-      // Let every copy this thread issued land before the CTA exits.
-      for (uint32_t i = it_k > kKVStages ? it_k - kKVStages : 0; i < it_k; ++i)
+      for (uint32_t i = n > kKVStages ? n - kKVStages : 0; i < n; ++i)
         drain_wait(&bars->k_full[i % kKVStages], (i / kKVStages) & 1);
-      for (uint32_t i = it_v > kKVStages ? it_v - kKVStages : 0; i < it_v; ++i)
-        drain_wait(&bars->v_full[i % kKVStages], (i / kKVStages) & 1);
       if (tc > 0) drain_wait(&bars->q_full, (tc - 1) & 1);
+    } else if (lane == 1) {  // V
+      prefetch_tmap(&tm_vc);
+      prefetch_tmap(&tm_vn);
+      uint32_t n = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
+        const Unit t = decode(a, tile);
+        for (int j = 0; ok && j < t.nb0; ++j) {
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && j >= t.nb1) break;
+            const int b = block_of(t, h, j);
+            const bool inA = b < t.nbA;
+            const int row = (inA ? b : b - t.nbA) * 128;
+            const uint32_t s = n % kKVStages, u = n / kKVStages;
+            if (!(ok = mbar_wait(&bars->v_empty[s], (u & 1) ^ 1, abort))) break;
+            mbar_expect_tx(&bars->v_full[s], kTileBytes);
+            tma_load_tile(sm + kOffV + s * kTileBytes, inA ? &tm_vc : &tm_vn, &bars->v_full[s],
+                          row, t.lh);
+            ++n;
+          }
+        }
+      }
+      for (uint32_t i = n > kKVStages ? n - kKVStages : 0; i < n; ++i)
+        drain_wait(&bars->v_full[i % kKVStages], (i / kKVStages) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t it = 0, tc = 0;
-      bool ok = true, pend = false, p_first = false;
-      uint32_t p_it = 0, p_tc = 0;
-      auto issue_pv = [&]() -> bool {
-        const uint32_t pb = p_it & 1, pu = p_it >> 1;
-        const uint32_t s = p_it % kKVStages, u = p_it / kKVStages;
-        if (p_first && !mbar_wait(&bars->o_free, (p_tc & 1) ^ 1, abort)) return false;
-        if (!mbar_wait(&bars->p_full[pb], pu & 1, abort)) return false;
-        if (!mbar_wait(&bars->v_full[s], u & 1, abort)) return false;
-        tc_fence_after();
-        const uint32_t vbase = smem_u32(sm + kOffV + s * kTileBytes);
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          mma_ts(tmem + kColO, tmem + kColP + pb * 64 + k * 8, mnmajor_desc(vbase, k), kIdescPV,
-                 (p_first && k == 0) ? 0u : 1u);
-        mma_commit(&bars->pv_done[pb]);
-        mma_commit(&bars->v_empty[s]);
-        return true;
-      };
+      uint32_t n = 0, uc = 0;
+      uint32_t p_use[2] = {0, 0};
+      bool ok = true;
       const uint32_t qbase = smem_u32(sm + kOffQ);
-      for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++tc) {
-        const Tile t = decode(a, tile);
-        if (!(ok = mbar_wait(&bars->q_full, tc & 1, abort))) break;
-        tc_fence_after();
-        for (int j = 0; j < t.nb; ++j, ++it) {
-          const uint32_t sb = it & 1, su = it >> 1;
-          const uint32_t s = it % kKVStages, u = it / kKVStages;
-          if (!(ok = mbar_wait(&bars->k_full[s], u & 1, abort))) break;
-          if (!(ok = mbar_wait(&bars->s_free[sb], (su & 1) ^ 1, abort))) break;
+      for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++uc) {
+        const Unit t = decode(a, tile);
+        const uint32_t base = n;
+        bool o_free_seen = false;
+        // O_h += P_h V for stream h's j-th block.
+        auto issue_pv = [&](int h, int j) -> bool {
+          if (!o_free_seen) {
+            if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort)) return false;
+            o_free_seen = true;
+          }
+          if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort)) return false;
+          ++p_use[h];
+          const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
+          const uint32_t s = pos % kKVStages, u = pos / kKVStages;
+          if (!mbar_wait(&bars->v_full[s], u & 1, abort)) return false;
           tc_fence_after();
-          const uint32_t kbase = smem_u32(sm + kOffK + s * kTileBytes);
+          const uint32_t vbase = smem_u32(sm + kOffV + s * kTileBytes);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ss(tmem + sb * 128, kmajor_desc(qbase, k), kmajor_desc(kbase, k), kIdescQK,
-                   k > 0 ? 1u : 0u);
-          mma_commit(&bars->s_full[sb]);
-          mma_commit(&bars->k_empty[s]);
-          if (j == t.nb - 1) mma_commit(&bars->q_empty);
-          if (pend && !(ok = issue_pv())) break;
-          pend = true;
-          p_it = it;
-          p_first = j == 0;
-          p_tc = tc;
+            mma_ts(tmem + col_o(h), tmem + col_s(h) + k * 8, mnmajor_desc(vbase, k), kIdescPV,
+                   (j == 0 && k == 0) ? 0u : 1u);
+          mma_commit(&bars->v_empty[s]);
+          return true;
+        };
+        if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort))) break;
+        tc_fence_after();
+        for (int j = 0; ok && j < t.nb0; ++j) {
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && j >= t.nb1) break;
+            if (j > 0 && !(ok = issue_pv(h, j - 1))) break;
+            const uint32_t s = n % kKVStages, u = n / kKVStages;
+            if (!(ok = mbar_wait(&bars->k_full[s], u & 1, abort))) break;
+            tc_fence_after();
+            const uint32_t kbase = smem_u32(sm + kOffK + s * kTileBytes);
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              mma_ss(tmem + col_s(h), kmajor_desc(qbase, k), kmajor_desc(kbase, k), kIdescQK,
+                     k > 0 ? 1u : 0u);
+            mma_commit(&bars->s_full[h]);
+            mma_commit(&bars->k_empty[s]);
+            ++n;
+          }
         }
+        if (!ok) break;
+        mma_commit(&bars->q_empty);  // every S of this unit issued
+        if (!(ok = issue_pv(0, t.nb0 - 1))) break;
+        if (t.nb1 > 0 && !(ok = issue_pv(1, t.nb1 - 1))) break;
+        mma_commit(&bars->o_ready);
       }
-      if (ok && pend) issue_pv();
       // Every MMA issued here completes before TMEM is released.
       mma_commit(&bars->mma_done);
       drain_wait(&bars->mma_done, 0);
     }
+  }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int row = (warp & 3) * 32 + lane;
-    const int half = warp >> 2;                 // key columns [64*half, 64*half + 64)
+    regs_increase<kSoftmaxRegs>();
+    // ------------------------------------------------------------ softmax warpgroups
+    const int h = warp >> 2;                    // stream
+    const int row = threadIdx.x & 127;          // query row = TMEM lane
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
-    const int quarter = warp & 3;               // rows shared by warps w and w+4
-    uint32_t it = 0, xc = 0;
+    const uint32_t tS = tmem + lane_addr + col_s(h);
+    uint32_t use = 0, base = 0, uc = 0;
     bool ok = true;
-    // Exchange of one float with the partner thread of the same row: round xc
-    // uses slot xc & 1; a slot is rewritten only two rounds later, after the
-    // partner has arrived on the round in between, i.e. after it read it.
-    auto exchange = [&](float v, float* other) -> bool {
-      const uint32_t slot = xc & 1;
-      bars->xval[slot][half][row] = v;
-      mbar_arrive(&bars->xbar[slot][quarter]);
-      if (!warp_wait(&bars->xbar[slot][quarter], (xc >> 1) & 1, abort)) return false;
-      *other = bars->xval[slot][half ^ 1][row];
-      ++xc;
-      return true;
-    };
-    for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
-      const Tile t = decode(a, tile);
+    for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++uc) {
+      const Unit t = decode(a, tile);
+      const int mine = h ? t.nb1 : t.nb0;
       float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < t.nb; ++j, ++it) {
-        const uint32_t sb = it & 1, su = it >> 1;
-        const bool inA = j < t.nbA;
-        const int64_t r0 = int64_t(inA ? j : j - t.nbA) * 128;
-        const int64_t rows_left = (inA ? t.nA : a.Lq) - r0;
-        const int nv_tile = rows_left < 128 ? int(rows_left) : 128;  // valid keys of the tile
-        const int nv = nv_tile - 64 * half < 0 ? 0 : (nv_tile - 64 * half > 64 ? 64 : nv_tile - 64 * half);
-        if (!(ok = warp_wait(&bars->s_full[sb], su & 1, abort))) break;
+      for (int j = 0; j < mine; ++j, ++use) {
+        const int b = block_of(t, h, j);
+        const bool inA = b < t.nbA;
+        const int64_t rows_left = (inA ? t.nA : a.Lq) - int64_t(inA ? b : b - t.nbA) * 128;
+        const int nv = rows_left < 128 ? int(rows_left) : 128;  // valid keys of the block
+        if (!(ok = warp_wait(&bars->s_full[h], use & 1, abort))) break;
         tc_fence_after();
-        uint32_t r[64];
-        tmem_ld32(tmem + lane_addr + sb * 128 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tmem + lane_addr + sb * 128 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        uint32_t sr[128];  // raw fp32 logits of this row
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
         tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->s_free[sb]);
-        float sv[64];
+        if (nv < 128) {  // ragged block: columns past the valid keys never count
 #pragma unroll
-        for (int i = 0; i < 64; ++i) sv[i] = __uint_as_float(r[i]);
-        if (nv < 64) {  // ragged tile: columns past the valid keys never count
-#pragma unroll
-          for (int i = 0; i < 64; ++i)
-            if (i >= nv) sv[i] = -INFINITY;
+          for (int i = 0; i < 128; ++i)
+            if (i >= nv) sr[i] = 0xff800000u;  // -inf
         }
-        float mx8[8];
+#define SV(i) __uint_as_float(sr[i])
+        float mx[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(sv[k], sv[k + 8]);
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(SV(k), SV(k + 8));
 #pragma unroll
-        for (int i = 16; i < 64; i += 16)
+        for (int i = 16; i < 128; i += 16)
 #pragma unroll
-          for (int k = 0; k < 8; ++k) mx8[k] = fmax3(mx8[k], sv[i + k], sv[i + k + 8]);
-        float pmax = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                           fmaxf(mx8[6], mx8[7]));
-        float omax;
-        if (!(ok = exchange(pmax, &omax))) break;
-        pmax = fmaxf(pmax, omax);
-        const float m_new = fmaxf(m, pmax * a.sl2);  // scale > 0
+          for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], SV(i + k), SV(i + k + 8));
+        const float bmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
+                                 fmaxf(mx[6], mx[7]));
+        const float m_new = fmaxf(m, bmax * a.sl2);  // scale > 0
         if (j == 0) {
           m = m_new;
         } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
-          // O holds blocks < j: wait for the last PV, then rescale this half in TMEM.
-          const uint32_t pi = it - 1;
-          if (!(ok = warp_wait(&bars->pv_done[pi & 1], (pi >> 1) & 1, abort))) break;
-          tc_fence_after();
+          // S_h of this block is complete, so the PV before it into O_h is too.
           const float alpha = ex2(m - m_new);
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + kColO + half * 64 + c * 32, o);
+#pragma unroll 1
+          for (int c = 0; c < 8; ++c) {
+            uint32_t o[16];
+            tmem_ld16(tmem + lane_addr + col_o(h) + c * 16, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem + lane_addr + kColO + half * 64 + c * 32, o);
+            for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st16(tmem + lane_addr + col_o(h) + c * 16, o);
           }
           tmem_st_wait();
           l *= alpha;
           m = m_new;
         }
-        // P_j into TMEM buffer pb once the PV that last read that buffer is done.
-        const uint32_t pb = it & 1, pu = it >> 1;
-        if (!(ok = warp_wait(&bars->pv_done[pb], (pu & 1) ^ 1, abort))) break;
-        tc_fence_after();
-        uint32_t pk[32];
-        float2 sum4[4];
+        float2 acc[4];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) sum4[k] = make_float2(0.f, 0.f);
+        for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
         const float2 sl2x2 = make_float2(a.sl2, a.sl2), negm2 = make_float2(-m, -m);
+        // P in two halves of 64 columns (32 packed TMEM columns each); P
+        // overwrites S columns whose values are already in registers.
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float2 e = ffma2(make_float2(sv[2 * i], sv[2 * i + 1]), sl2x2, negm2);
-          const float2 p = make_float2(ex2(e.x), ex2(e.y));
-          sum4[i & 3] = fadd2(sum4[i & 3], p);
-          pk[i] = pack_bf16(p.x, p.y);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int c = 64 * hh + 2 * i;
+            const float2 e = ffma2(make_float2(SV(c), SV(c + 1)), sl2x2, negm2);
+            const float2 p = (i & 3) == 3 ? exp2_poly2(e) : make_float2(ex2(e.x), ex2(e.y));
+            acc[i & 3] = fadd2(acc[i & 3], p);
+            pk[i] = pack_bf16(p.x, p.y);
+          }
+          tmem_st32(tS + 32 * hh, pk);
         }
-        const float2 s2 = fadd2(fadd2(sum4[0], sum4[1]), fadd2(sum4[2], sum4[3]));
+#undef SV
+        const float2 s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
         l += s2.x + s2.y;
-        tmem_st32(tmem + lane_addr + kColP + pb * 64 + half * 32, pk);
         tmem_st_wait();
-        if (nv_tile < 128) {
+        if (nv < 128) {
           // V rows past the valid keys may hold anything (P is 0 there, but
           // 0 * NaN is not 0): zero them before the PV MMA reads the stage.
-          const uint32_t s = it % kKVStages, u = it / kKVStages;
+          const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
+          const uint32_t s = pos % kKVStages, u = pos / kKVStages;
           if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort))) break;
-          if (row >= nv_tile) {
-            uint4* v = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + half * kRegionBytes + row * 128);
+          if (row >= nv) {
+            uint4* v0 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + row * 128);
+            uint4* v1 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + kRegionBytes + row * 128);
             const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) v[c] = z;
+            for (int c = 0; c < 8; ++c) {
+              v0[c] = z;
+              v1[c] = z;
+            }
           }
           fence_proxy_async_smem();
         }
         tc_fence_before();
-        mbar_arrive(&bars->p_full[pb]);
+        mbar_arrive(&bars->p_full[h]);
       }
       if (!ok) break;
-      // Epilogue: O / l -> bf16 -> out, each thread its 64 columns.
-      const uint32_t last = it - 1;
-      if (!(ok = warp_wait(&bars->pv_done[last & 1], (last >> 1) & 1, abort))) break;
+      base += uint32_t(t.nb);
+      // ---- merge the two streams and write this thread's 64 output columns
+      if (!(ok = warp_wait(&bars->o_ready, uc & 1, abort))) break;
       tc_fence_after();
-      uint32_t o[64];
-      tmem_ld32(tmem + lane_addr + kColO + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-      tmem_ld32(tmem + lane_addr + kColO + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->o_free);
-      float ol;
-      if (!(ok = exchange(l, &ol))) break;
-      const float inv = 1.f / (l + ol);
+      if (!(ok = warp_wait(&bars->x_read, (uc & 1) ^ 1, abort))) break;  // last unit's reads done
+      bars->xml[h][row] = make_float2(m, l);
+      mbar_arrive(&bars->x_full);
+      if (!(ok = warp_wait(&bars->x_full, uc & 1, abort))) break;
+      const float2 other = bars->xml[h ^ 1][row];
+      mbar_arrive(&bars->x_read);
+      const float m0 = h ? other.x : m, l0 = h ? other.y : l;
+      const float m1 = h ? m : other.x, l1 = h ? l : other.y;
+      const bool two = t.nb1 > 0;
+      const float M = two ? fmaxf(m0, m1) : m0;
+      const float a0 = ex2(m0 - M), a1 = two ? ex2(m1 - M) : 0.f;
+      const float inv = 1.f / (l0 * a0 + (two ? l1 * a1 : 0.f));
+      const float c0 = a0 * inv, c1 = a1 * inv;
+      // 64 columns per thread, merged and written 32 at a time.
       const int64_t q = int64_t(t.qt) * 128 + row;
-      if (q < a.Lq) {
-        uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t(t.lh) * a.Lq + q) * 128 + half * 64);
+      uint4* dst = reinterpret_cast<uint4*>(a.out + (int64_t(t.lh) * a.Lq + q) * 128 + h * 64);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 v;
-          v.x = pack_bf16(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-          v.y = pack_bf16(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-          v.z = pack_bf16(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-          v.w = pack_bf16(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-          dst[c] = v;
+      for (int c = 0; c < 2; ++c) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(tmem + lane_addr + col_o(0) + h * 64 + c * 32, r0);
+        if (two) tmem_ld32(tmem + lane_addr + col_o(1) + h * 64 + c * 32, r1);
+        tmem_ld_wait();
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0 = __uint_as_float(r0[2 * i]) * c0, x1 = __uint_as_float(r0[2 * i + 1]) * c0;
+          if (two) {
+            x0 = fmaf(__uint_as_float(r1[2 * i]), c1, x0);
+            x1 = fmaf(__uint_as_float(r1[2 * i + 1]), c1, x1);
+          }
+          w[i] = pack_bf16(x0, x1);
+        }
+        if (q < a.Lq) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            dst[c * 4 + k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(&bars->o_free);
     }
   }
 
@@ -406,6 +474,19 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_dealloc(tmem, 512);
   }
   if (threadIdx.x == 0 && bars->abort) report(a.status, FKV_ERR_TIMEOUT, blockIdx.x);
+}
+
+// Evaluates the attention kernel's FMA-pipe exp2 on an array (for testing it
+// against the hardware exp2 and its error bound).
+__global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict__ y, int64_t n) {
+  const int64_t i = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
 }
 
 }  // namespace sm100
@@ -448,6 +529,13 @@ cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_
   if (e != cudaSuccess) return e;
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();
   attend_sm100_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(tq, tkc, tvc, tkn, tvn, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t pairs = (n + 1) / 2;
+  sm100::exp2_poly_kernel<<<unsigned((pairs + 255) / 256), 256, 0, s>>>(x, y, n);
   return cudaGetLastError();
 }
 

@@ -240,6 +240,12 @@ int32_t fkv_step_launches(const fkv_params_t* p, int32_t* launches) {
   return FKV_OK;
 }
 
+int32_t fkv_exp2_emulated(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0) return FKV_ERR_SHAPE;
+  if (n > 0 && (!x || !y)) return FKV_ERR_INVALID_ARG;
+  return cuda_status(launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t fkv_workspace_init(void* ws, size_t bytes, void* stream) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < 256) return FKV_ERR_WORKSPACE;
   return cuda_status(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));

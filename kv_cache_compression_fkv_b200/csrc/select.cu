@@ -84,34 +84,22 @@ cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uin
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 
-// Exclusive block-wide prefix count of `flag` in thread order, plus the total.
-__device__ __forceinline__ int block_excl_count(bool flag, int* warp_tot, int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned b = __ballot_sync(0xffffffffu, flag);
-  if (lane == 0) warp_tot[warp] = __popc(b);
-  __syncthreads();
-  int base = 0, tot = 0;
-  for (int w = 0; w < kSelWarps; ++w) {
-    const int c = warp_tot[w];
-    base += (w < warp) ? c : 0;
-    tot += c;
-  }
-  __syncthreads();
-  *total = tot;
-  return base + __popc(b & ((1u << lane) - 1u));
-}
+// Keys cached in shared memory when they fit (the 14B workload's 18720
+// candidates take 73 KB); otherwise every pass re-reads them (from L2).
+constexpr int64_t kSelCacheKeys = 40960;
 
 __global__ void __launch_bounds__(kSelThreads)
-select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N,
+select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
                     const float* __restrict__ phi, const int32_t* __restrict__ k_per_head,
                     int32_t* __restrict__ kept_idx, int32_t* __restrict__ kept_cnt,
                     int32_t* status) {
+  extern __shared__ uint32_t skeys[];
   __shared__ unsigned hist[256];
   __shared__ int warp_tot[kSelWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int64_t s_need;
   const int lh = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* ph = phi + int64_t(lh) * n_c;
   int32_t* out = kept_idx + int64_t(lh) * N;
   int64_t C = k_per_head[lh];
@@ -123,28 +111,59 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N,
   for (int64_t i = tid; i < R; i += kSelThreads) out[S + C + i] = int32_t(N - R + i);
   if (tid == 0) kept_cnt[lh] = int32_t(S + C + R);
   if (C == 0) return;
+  if (cached) {
+    for (int64_t j = tid; j < n_c; j += kSelThreads) skeys[j] = ordered_key(ph[j]);
+    __syncthreads();
+  }
+  auto key_at = [&](int64_t j) -> uint32_t { return cached ? skeys[j] : ordered_key(ph[j]); };
 
-  // Radix select of the C-th largest key, most significant byte first.
+  // Radix select of the C-th largest key, most significant byte first.  Lanes
+  // of a warp that hit the same bin are merged (__match_any_sync) into one
+  // shared-memory atomic, so clustered scores do not serialise the histogram.
   uint32_t prefix = 0, pmask = 0;
   int64_t need = C;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
     __syncthreads();
-    for (int64_t j = tid; j < n_c; j += kSelThreads) {
-      const uint32_t key = ordered_key(ph[j]);
-      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    for (int64_t base = int64_t(warp) * 32; base < n_c; base += kSelThreads) {
+      const int64_t j = base + lane;
+      uint32_t bin = 256;  // no bin
+      if (j < n_c) {
+        const uint32_t key = key_at(j);
+        if ((key & pmask) == prefix) bin = (key >> shift) & 255u;
+      }
+      const unsigned grp = __match_any_sync(0xffffffffu, bin);
+      if (bin < 256 && lane == __ffs(grp) - 1) atomicAdd(&hist[bin], unsigned(__popc(grp)));
     }
     __syncthreads();
-    if (tid == 0) {
-      int64_t above = 0;
-      int b = 255;
-      for (; b > 0; --b) {
-        if (above + int64_t(hist[b]) >= need) break;
-        above += hist[b];
+    if (warp == 0) {
+      // Lane l owns bins 8*(31-l) .. 8*(31-l)+7 (lane 0 the highest); a warp
+      // inclusive scan from the top finds the bin where the count of larger
+      // keys first reaches `need`.
+      const int b0 = 8 * (31 - lane);
+      unsigned cnt = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cnt += hist[b0 + k];
+      unsigned incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
       }
-      s_prefix = prefix | (uint32_t(b) << shift);
-      s_need = need - above;
+      const unsigned excl = incl - cnt;
+      const bool here = int64_t(excl) < need && int64_t(incl) >= need;
+      const unsigned who = __ballot_sync(0xffffffffu, here);
+      if (lane == __ffs(who) - 1) {
+        int64_t above = excl;
+        int b = b0 + 7;
+        for (; b > b0; --b) {
+          if (above + int64_t(hist[b]) >= need) break;
+          above += hist[b];
+        }
+        s_prefix = prefix | (uint32_t(b) << shift);
+        s_need = need - above;
+      }
     }
     __syncthreads();
     prefix = s_prefix;
@@ -153,28 +172,49 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N,
     __syncthreads();
   }
   const uint32_t t = prefix;  // exact key of the C-th largest score
-  // Stable compaction: keys > t, then the first `need` keys == t by index.
-  int64_t base = 0, eq_seen = 0;
+  // Stable compaction in index order: every key > t, and the first `need`
+  // keys == t.  Before position j, gt_before keys > t and eq_before keys == t
+  // occur, of which min(eq_before, need) are taken, so one scan of the
+  // packed pair (gt, eq) per chunk gives every destination.
+  int64_t gt_seen = 0, eq_seen = 0;
   for (int64_t c0 = 0; c0 < n_c; c0 += kSelThreads) {
     const int64_t j = c0 + tid;
-    const uint32_t key = j < n_c ? ordered_key(ph[j]) : 0u;
+    const uint32_t key = j < n_c ? key_at(j) : 0u;
     const bool gt = j < n_c && key > t;
     const bool eq = j < n_c && key == t;
-    int eq_tot, take_tot;
-    const int eq_rank = block_excl_count(eq, warp_tot, &eq_tot);
-    const bool take = gt || (eq && eq_seen + eq_rank < need);
-    const int pos = block_excl_count(take, warp_tot, &take_tot);
-    if (take) out[S + base + pos] = int32_t(S + j);
-    base += take_tot;
-    eq_seen += eq_tot;
+    const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    if (lane == 0) warp_tot[warp] = int(__popc(bg) | (__popc(be) << 16));
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      const int c = warp_tot[w];
+      before += (w < warp) ? c : 0;
+      total += c;
+    }
+    __syncthreads();
+    const unsigned below = (1u << lane) - 1u;
+    const int64_t gt_before = gt_seen + (before & 0xFFFF) + __popc(bg & below);
+    const int64_t eq_before = eq_seen + (before >> 16) + __popc(be & below);
+    if (gt || (eq && eq_before < need)) {
+      const int64_t pos = gt_before + (eq_before < need ? eq_before : need);
+      out[S + pos] = int32_t(S + j);
+    }
+    gt_seen += total & 0xFFFF;
+    eq_seen += total >> 16;
   }
 }
 
 cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int32_t* k_per_head,
                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                 cudaStream_t s) {
-  select_token_kernel<<<d.LH, kSelThreads, 0, s>>>(d.nseg, d.S, d.R, d.N, seg_score, k_per_head,
-                                                   kept_idx, kept_cnt, status);
+  const int cached = d.nseg <= kSelCacheKeys;
+  const size_t smem = cached ? sizeof(uint32_t) * size_t(d.nseg > 0 ? d.nseg : 1) : 0;
+  cudaError_t e = cudaFuncSetAttribute(select_token_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(sizeof(uint32_t) * kSelCacheKeys));
+  if (e != cudaSuccess) return e;
+  select_token_kernel<<<d.LH, kSelThreads, smem, s>>>(d.nseg, d.S, d.R, d.N, cached, seg_score,
+                                                      k_per_head, kept_idx, kept_cnt, status);
   return cudaGetLastError();
 }
 

@@ -1,5 +1,5 @@
 // CUDA-core (SIMT) kernels: fp32 path of segment scoring and of attention,
-// the finalisation of the segment mass, and the token-variant scoring.
+// and the finalisation of the segment mass (both dtypes).
 //
 // Frame-mode segment mass (Forcing-KV, ai-feeds.com/i/paper/2605.09681,
 // "关键模块" 3), computed in one pass over the history keys:
@@ -168,89 +168,6 @@ cudaError_t launch_score_frame_finalize(const Dims& d, const uint8_t* head_role,
   score_rows_kernel<<<g1, 256, 0, s>>>(d.F, d.n_s, head_role, part_ml, row_ml);
   dim3 g2(unsigned(d.F), unsigned(d.LH));
   score_mass_kernel<<<g2, 256, 0, s>>>(d.F, d.n_s, head_role, part_ml, row_ml, seg_score);
-  return cudaGetLastError();
-}
-
-// ---------------------------------------------------------------------------
-// Token variant (Deep Forcing, bxzpzcl.cn/news/2125000, section 3.1 step 2):
-// phi_j = sum_r q_r . k_j = (sum_r q_r) . k_j.  First qbar = sum_r q_r in fp32
-// (8 row groups per dim, combined in a fixed order), then one dot product per
-// candidate row: a GEMV bound by reading the candidate keys once.
-
-template <typename T>
-__global__ void qsum_kernel(int D, int64_t n_q, const T* __restrict__ q_score,
-                            float* __restrict__ qbar) {
-  __shared__ float part[8][kDMax];
-  const int lh = blockIdx.x;
-  const int d = threadIdx.x % kDMax, g = threadIdx.x / kDMax;
-  float acc = 0.f;
-  if (d < D) {
-    const T* q = q_score + int64_t(lh) * n_q * D + d;
-    for (int64_t r = g; r < n_q; r += 8) acc += to_f32(q[r * D]);
-  }
-  part[g][d] = acc;
-  __syncthreads();
-  if (g == 0 && d < D) {
-    float tot = 0.f;
-    for (int k = 0; k < 8; ++k) tot += part[k][d];
-    qbar[int64_t(lh) * D + d] = tot;
-  }
-}
-
-// One warp per candidate row, lanes over D in 4-element groups.
-template <typename T>
-__global__ void phi_kernel(int D, int64_t N, int64_t S, int64_t n_c, const T* __restrict__ k_hist,
-                           const float* __restrict__ qbar, float* __restrict__ phi) {
-  const int lh = blockIdx.y;
-  const int lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
-  const int q4 = D / 4;
-  float qb[4] = {0.f, 0.f, 0.f, 0.f};
-  if (lane < q4)
-    for (int t = 0; t < 4; ++t) qb[t] = qbar[int64_t(lh) * D + lane * 4 + t];
-  const T* kc = k_hist + (int64_t(lh) * N + S) * D;
-  for (int64_t j = int64_t(blockIdx.x) * warps + (threadIdx.x >> 5); j < n_c;
-       j += int64_t(gridDim.x) * warps) {
-    float acc = 0.f;
-    if (lane < q4) {
-      const T* p = kc + j * D + lane * 4;
-      float x[4];
-      if constexpr (sizeof(T) == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(p);
-        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-      } else {
-        const uint2 v = *reinterpret_cast<const uint2*>(p);
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
-        x[0] = __low2float(a); x[1] = __high2float(a); x[2] = __low2float(b); x[3] = __high2float(b);
-      }
-      for (int t = 0; t < 4; ++t) acc = fmaf(qb[t], x[t], acc);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) phi[int64_t(lh) * n_c + j] = acc;
-  }
-}
-
-cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
-                               float* qbar, float* seg_score, cudaStream_t s) {
-  if (d.bf16)
-    qsum_kernel<__nv_bfloat16><<<d.LH, 8 * kDMax, 0, s>>>(
-        d.D, d.n_score_q, static_cast<const __nv_bfloat16*>(q_score), qbar);
-  else
-    qsum_kernel<float><<<d.LH, 8 * kDMax, 0, s>>>(d.D, d.n_score_q,
-                                                  static_cast<const float*>(q_score), qbar);
-  const int warps = 8;
-  int64_t bx = (d.nseg + warps - 1) / warps;
-  if (bx > 4096) bx = 4096;
-  dim3 grid(unsigned(bx), unsigned(d.LH));
-  if (d.bf16)
-    phi_kernel<__nv_bfloat16><<<grid, warps * 32, 0, s>>>(
-        d.D, d.N, d.S, d.nseg, static_cast<const __nv_bfloat16*>(k_hist), qbar, seg_score);
-  else
-    phi_kernel<float><<<grid, warps * 32, 0, s>>>(d.D, d.N, d.S, d.nseg,
-                                                  static_cast<const float*>(k_hist), qbar,
-                                                  seg_score);
   return cudaGetLastError();
 }
 

@@ -50,6 +50,15 @@ def test_empty_history(cuda_device):
     parity.check_step(w, x, res)
 
 
+@pytest.mark.parametrize("T,F", [(96, 0), (40, 2), (128, 1)])
+def test_few_key_blocks(cuda_device, T, F):
+    """One or two 128-key blocks in total (one attention stream may be empty)."""
+    w = _small(T=T, F=F, Fc=1, static_frames=tuple(range(F)), k_dynamic=F)
+    x = wl.generate(w)
+    res = parity.run_step(w, x, comp_rows=max(F * T, 0))
+    parity.check_step(w, x, res)
+
+
 def test_zero_pruning_is_full_attention_and_bit_identical(cuda_device):
     """mask = every frame, k = F: the output equals full attention over
     history + chunk, and is bit-identical to attending the raw history."""

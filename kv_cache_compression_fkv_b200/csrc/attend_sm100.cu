@@ -23,8 +23,9 @@
 //              - m) as bf16 pairs into the first 64 columns of S_h, and
 //              rescales O_h in TMEM only when m grows by more than 2^8 (lazy
 //              rescaling: P stays <= 256, exact after the final merge).
-//              Three of every four exponential pairs go to the MUFU unit, one
-//              to an FMA-pipe polynomial (exp2_poly2) to balance the pipes.
+//              Exponentials run on the MUFU unit; FKV_POLY_EVERY = n sends
+//              one pair in n to the FMA-pipe polynomial exp2_poly2 instead
+//              (measured slower at 480P, where MUFU is ~45% busy: default 0).
 //   warp 8     TMA: lane 0 loads Q (once per unit) and the K blocks, lane 1
 //              the V blocks, into 3-stage rings in the order the MMAs use
 //              them: stream 0 block j, stream 1 block j, stream 0 block j+1...
@@ -66,6 +67,10 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 128, true);
 constexpr float kRescaleLog2 = 8.0f;
+// One of every FKV_POLY_EVERY exponential pairs goes to the FMA-pipe exp2 (0: none).
+#ifndef FKV_POLY_EVERY
+#define FKV_POLY_EVERY 0
+#endif
 
 __host__ __device__ constexpr uint32_t col_s(int h) { return 128u * uint32_t(h); }
 __host__ __device__ constexpr uint32_t col_o(int h) { return 256u + 128u * uint32_t(h); }
@@ -389,7 +394,10 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           for (int i = 0; i < 32; ++i) {
             const int c = 64 * hh + 2 * i;
             const float2 e = ffma2(make_float2(SV(c), SV(c + 1)), sl2x2, negm2);
-            const float2 p = (i & 3) == 3 ? exp2_poly2(e) : make_float2(ex2(e.x), ex2(e.y));
+            const float2 p = (FKV_POLY_EVERY > 0 && i % (FKV_POLY_EVERY > 0 ? FKV_POLY_EVERY : 1) ==
+                                                       (FKV_POLY_EVERY > 0 ? FKV_POLY_EVERY : 1) - 1)
+                                 ? exp2_poly2(e)
+                                 : make_float2(ex2(e.x), ex2(e.y));
             acc[i & 3] = fadd2(acc[i & 3], p);
             pk[i] = pack_bf16(p.x, p.y);
           }

@@ -17,7 +17,7 @@ WsLayout ws_layout(const Dims& d) {
   w.part_ml = w.row_ml = w.qbar = off;
   if (!d.token) {
     w.part_ml = off;
-    off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(d.F) * size_t(d.n_s));
+    off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(d.F) * kScoreSplit * size_t(d.n_s));
     w.row_ml = off;
     off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(d.n_s));
   } else {
@@ -127,7 +127,8 @@ static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, c
                                                     status_ptr(ws), s)
                          : launch_score_frame_simt(d, q_cur, k_hist, head_role, part, s);
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(launch_score_frame_finalize(d, head_role, part, rows, seg_score, s));
+  return cuda_status(
+      launch_score_frame_finalize(d, d.bf16 ? kScoreSplit : 1, head_role, part, rows, seg_score, s));
 }
 
 static int32_t do_select(const Dims& d, const float* seg_score, const uint8_t* head_role,
@@ -161,7 +162,7 @@ static int32_t do_attend(const Dims& d, const void* q_cur, const void* k_cur, co
 static int32_t step_launch_count(const Dims& d) {
   int32_t n = 0;
   if (d.token) n += d.nseg > 0 ? 2 : 0;   // q-sum, phi
-  else n += d.F > 0 ? 3 : 0;              // partial, row merge, mass
+  else n += d.F > 0 ? 2 : 0;              // partial statistics, finalize
   n += 1;                                 // select
   n += 1;                                 // gather
   n += 1;                                 // attention

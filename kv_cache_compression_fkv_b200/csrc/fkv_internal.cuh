@@ -29,10 +29,14 @@ struct Dims {
   int elem;          // bytes per activation element
 };
 
+// Sub-segments per frame of the tensor-core scoring kernel (the CUDA-core
+// scoring produces one per frame).
+constexpr int kScoreSplit = 2;
+
 // Workspace layout (byte offsets from the workspace base, 256-B aligned).
 struct WsLayout {
   size_t status;     // int32[2]: first device error, detail
-  size_t part_ml;    // frame mode: float2 [LH][F][n_s] per-frame (max, sumexp)
+  size_t part_ml;    // frame mode: float2 [LH][F*kScoreSplit][n_s] per-sub-segment (max, sum)
   size_t row_ml;     // frame mode: float2 [LH][n_s] per-row (max, sum)
   size_t qbar;       // token mode: float [LH][D] summed scoring queries
   size_t total;
@@ -64,7 +68,7 @@ __device__ __forceinline__ uint32_t ordered_key(float x) {
 // ---- launchers (each returns cudaGetLastError() of its launches) ----------
 cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
                                     const uint8_t* head_role, float2* part_ml, cudaStream_t s);
-cudaError_t launch_score_frame_finalize(const Dims& d, const uint8_t* head_role,
+cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
                                         const float2* part_ml, float2* row_ml, float* seg_score,
                                         cudaStream_t s);
 cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,

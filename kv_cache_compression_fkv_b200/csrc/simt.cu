@@ -102,47 +102,58 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
   if (c8 == 0 && r < nq) part_ml[(int64_t(lh) * F + f) * n_s + row0 + r] = make_float2(m, l);
 }
 
-// Per-row merge of the frame partials.  grid = (ceil(n_s / 256), L*H).
-__global__ void score_rows_kernel(int F, int64_t n_s, const uint8_t* __restrict__ head_role,
-                                  const float2* __restrict__ part_ml, float2* __restrict__ row_ml) {
-  const int lh = blockIdx.y;
-  const int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (!head_role[lh] || i >= n_s) return;
-  const float2* p = part_ml + int64_t(lh) * F * n_s + i;
-  float M = -INFINITY;
-  for (int f = 0; f < F; ++f) M = fmaxf(M, p[int64_t(f) * n_s].x);
-  float Ls = 0.f;
-  for (int f = 0; f < F; ++f) {
-    const float2 ml = p[int64_t(f) * n_s];
-    Ls += ml.y * exp2f(ml.x - M);
-  }
-  row_ml[int64_t(lh) * n_s + i] = make_float2(M, Ls);
-}
+// Frame masses from the partial statistics of G = F*split sub-segments per
+// head (split consecutive sub-segments per frame).  One CTA per (layer, head):
+//   row merge   M_i = max_g m_{g,i},  L_i = sum_g l_{g,i} 2^(m_{g,i} - M_i)
+//               (stored as (M_i, 1/L_i) in row_ml),
+//   frame mass  mass_f = sum_i sum_{g in f} l_{g,i} 2^(m_{g,i} - M_i) / L_i,
+// each warp owning frames f = warp, warp + 8, ..., lanes striding the rows,
+// then a fixed shuffle tree: the order of every sum is fixed (deterministic).
+constexpr int kFinThreads = 1024;
 
-// mass_f = sum_i l_{f,i} 2^(m_{f,i} - M_i) / L_i.  grid = (F, L*H), 256 threads.
-__global__ void score_mass_kernel(int F, int64_t n_s, const uint8_t* __restrict__ head_role,
-                                  const float2* __restrict__ part_ml,
-                                  const float2* __restrict__ row_ml, float* __restrict__ seg_score) {
-  __shared__ float red[256];
-  const int lh = blockIdx.y, f = blockIdx.x;
+__global__ void __launch_bounds__(kFinThreads)
+score_finalize_kernel(int F, int split, int64_t n_s, const uint8_t* __restrict__ head_role,
+                      const float2* __restrict__ part_ml, float2* __restrict__ row_ml,
+                      float* __restrict__ seg_score) {
+  const int lh = blockIdx.x;
+  const int G = F * split;
+  float* out = seg_score + int64_t(lh) * F;
   if (!head_role[lh]) {
-    if (threadIdx.x == 0) seg_score[int64_t(lh) * F + f] = 0.f;
+    for (int f = threadIdx.x; f < F; f += blockDim.x) out[f] = 0.f;
     return;
   }
-  const float2* p = part_ml + (int64_t(lh) * F + f) * n_s;
-  const float2* rm = row_ml + int64_t(lh) * n_s;
-  float acc = 0.f;
-  for (int64_t i = threadIdx.x; i < n_s; i += 256) {
-    const float2 ml = p[i], MR = rm[i];
-    acc += ml.y * exp2f(ml.x - MR.x) / MR.y;
+  const float2* p = part_ml + int64_t(lh) * G * n_s;
+  float2* rm = row_ml + int64_t(lh) * n_s;
+  for (int64_t i = threadIdx.x; i < n_s; i += blockDim.x) {
+    float M = -INFINITY;
+#pragma unroll 8
+    for (int g = 0; g < G; ++g) M = fmaxf(M, p[int64_t(g) * n_s + i].x);
+    float Ls = 0.f;
+#pragma unroll 8
+    for (int g = 0; g < G; ++g) {
+      const float2 ml = p[int64_t(g) * n_s + i];
+      if (ml.y != 0.f) Ls += ml.y * exp2f(ml.x - M);
+    }
+    rm[i] = make_float2(M, 1.f / Ls);
   }
-  red[threadIdx.x] = acc;
   __syncthreads();
-  for (int w = 128; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-    __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int f = warp; f < F; f += blockDim.x >> 5) {
+    float acc = 0.f;
+#pragma unroll 4
+    for (int64_t i = lane; i < n_s; i += 32) {
+      const float2 MR = rm[i];
+      float t = 0.f;
+      for (int s = 0; s < split; ++s) {
+        const float2 ml = p[int64_t(f * split + s) * n_s + i];
+        if (ml.y != 0.f) t += ml.y * exp2f(ml.x - MR.x);
+      }
+      acc += t * MR.y;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) out[f] = acc;
   }
-  if (threadIdx.x == 0) seg_score[int64_t(lh) * F + f] = red[0];
 }
 
 cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
@@ -161,13 +172,11 @@ cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void
   return cudaGetLastError();
 }
 
-cudaError_t launch_score_frame_finalize(const Dims& d, const uint8_t* head_role,
+cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
                                         const float2* part_ml, float2* row_ml, float* seg_score,
                                         cudaStream_t s) {
-  dim3 g1(unsigned((d.n_s + 255) / 256), unsigned(d.LH));
-  score_rows_kernel<<<g1, 256, 0, s>>>(d.F, d.n_s, head_role, part_ml, row_ml);
-  dim3 g2(unsigned(d.F), unsigned(d.LH));
-  score_mass_kernel<<<g2, 256, 0, s>>>(d.F, d.n_s, head_role, part_ml, row_ml, seg_score);
+  score_finalize_kernel<<<d.LH, kFinThreads, 0, s>>>(d.F, split, d.n_s, head_role, part_ml,
+                                                     row_ml, seg_score);
   return cudaGetLastError();
 }
 

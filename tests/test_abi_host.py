@@ -94,7 +94,7 @@ def test_derived_sizes(lib):
     s = fkv.sizes(_p())
     assert s["nseg"] == 6 and s["max_kept"] == 6 and s["max_comp_rows"] == 192
     # status block + (max, sum) per frame and scoring row + (max, sum) per row
-    assert s["ws_bytes"] == 256 + 4 * 6 * 32 * 8 + 4 * 32 * 8
+    assert s["ws_bytes"] == 256 + 4 * 6 * 2 * 32 * 8 + 4 * 32 * 8  # 2 sub-segments per frame
     t = fkv.sizes(_p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8))
     assert t["nseg"] == 192 - 80 and t["max_kept"] == 192 and t["max_comp_rows"] == 192
 

@@ -166,6 +166,30 @@ def committed_traffic(kernel_key, workload, src_hash):
     return e.get("dram_bytes_per_launch")
 
 
+def replica_workload(w, rank, world):
+    """Weak scaling with replicas: rank r runs the same workload shape on its
+    own independent inputs (seeds offset by rank); there is no exchange."""
+    if world <= 1:
+        return w
+    return wl.scaled(w, seed=w.seed + 7919 * rank, layer_seeds=None if w.layer_seeds is None else
+                     tuple(s + 7919 * rank for s in w.layer_seeds))
+
+
+def max_over_ranks(value, dist=None, device=None):
+    """Max of a per-rank float over the process group (the job's time is its
+    slowest rank's)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(units_per_rank, world, max_ms):
+    """Whole-job throughput: units processed by all ranks / slowest rank's time."""
+    return units_per_rank * world / (max_ms / 1e3)
+
+
 def run_ours(args, rank, world, local_rank):
     import kv_cache_compression_fkv_b200 as fkv
     dist = None
@@ -175,10 +199,7 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
-    w = wl.get(args.workload)
-    if world > 1:  # independent problem per rank (replicas)
-        w = wl.scaled(w, seed=w.seed + 7919 * rank, layer_seeds=None if w.layer_seeds is None else
-                      tuple(s + 7919 * rank for s in w.layer_seeds))
+    w = replica_workload(wl.get(args.workload), rank, world)
     x_cpu = wl.generate(w)
     p = fkv.params_for(w)
     stream = torch.cuda.current_stream(dev)
@@ -191,13 +212,6 @@ def run_ours(args, rank, world, local_rank):
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
-
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     # warm-up
     for _ in range(args.warmup):
@@ -220,7 +234,7 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize(dev)
     barrier()
     step_ms = [a.elapsed_time(b) for a, b in evs]
-    total_ms = max_over_ranks(sum(step_ms))
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     clocks = clk.summary()
 
     # ---- per-kernel breakdown: the same kernels through the four entry points
@@ -293,7 +307,7 @@ def run_ours(args, rank, world, local_rank):
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end))
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dist, dev)
     for b in range(2):
         st, det = fkv.read_status(os_[b]["ws"])
         if st != 0:
@@ -305,9 +319,8 @@ def run_ours(args, rank, world, local_rank):
     alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
                       else torch.ones(w.L, w.H))
     peaks, peak_kind = load_peaks()
-    units = w.L * args.steps * world
-    value = units / (total_ms / 1e3)
-    e2e_value = units / (e2e_ms / 1e3)
+    value = aggregate_throughput(w.L * args.steps, world, total_ms)
+    e2e_value = aggregate_throughput(w.L * args.steps, world, e2e_ms)
     attn_tfs = alg["attn_flops"] / (part["attend"] * 1e-3) / 1e12
     gather_gbs = alg["gather_bytes"] / (part["gather"] * 1e-3) / 1e9
     score_tfs = alg["score_flops"] / (part["score"] * 1e-3) / 1e12

@@ -316,6 +316,48 @@ def run_ours(args, rank, world, local_rank):
     if st != 0:
         raise RuntimeError(f"device status {st} on head {det}")
 
+    # ---- chunk lifecycle: kDenoise denoising steps of one chunk, then the cache
+    # advance (next history = the most recent kept frames + the chunk).  Two
+    # policies: compress at every denoising step, or once per chunk and reuse
+    # the selection (attention alone for the later steps).
+    lifecycle = None
+    if w.granularity == "frame" and w.L == 1:
+        n_den = 4
+        kept = int(outs["kept_cnt"].min())
+        window = min(kept, w.F - w.Fc) + w.Fc
+        k_next = torch.empty((w.L, w.H, window * w.T, w.D), dtype=x["k_cur"].dtype, device=dev)
+        v_next = torch.empty_like(k_next)
+
+        def advance():
+            fkv.cache_advance(p, outs["k_comp"], outs["v_comp"], outs["kept_cnt"], x["k_cur"],
+                              x["v_cur"], window, k_next, v_next, outs["ws"])
+
+        def attend_only():
+            fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"],
+                                  outs["v_comp"], outs["kept_cnt"], outs["out"], outs["ws"])
+
+        def timed(body):
+            evs_ = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)]
+            for i in range(args.steps):
+                flush.fill_(i & 0xFF)
+                evs_[i][0].record(stream)
+                body()
+                evs_[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            return statistics.mean(a_.elapsed_time(b_) for a_, b_ in evs_)
+
+        every = timed(lambda: ([fkv.step(p, x, outs, io=io) for _ in range(n_den)], advance()))
+        reuse = timed(lambda: (fkv.step(p, x, outs, io=io),
+                               [attend_only() for _ in range(n_den - 1)], advance()))
+        lifecycle = {"denoising_steps": n_den, "window_frames": window,
+                     "ms_per_chunk_compress_every_step": round(every, 4),
+                     "ms_per_chunk_compress_once": round(reuse, 4),
+                     "chunks_per_s_compress_once": round(1e3 / reuse, 2)}
+        st, det = fkv.read_status(outs["ws"])
+        if st != 0:
+            raise RuntimeError(f"device status {st} on head {det}")
+
     alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
                       else torch.ones(w.L, w.H))
     peaks, peak_kind = load_peaks()
@@ -366,6 +408,8 @@ def run_ours(args, rank, world, local_rank):
         "kernels": kernels,
         "clocks": clocks,
     }
+    if lifecycle is not None:
+        line["lifecycle"] = lifecycle
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget)
     if dist is not None:

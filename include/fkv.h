@@ -229,6 +229,28 @@ int32_t fkv_attend_compressed(const fkv_params_t* p, const void* q_cur, const vo
                               const void* v_cur, const void* k_comp, const void* v_comp,
                               const int32_t* kept_cnt, void* out, void* ws, void* stream);
 
+/* Cache lifecycle: the history cache for the next chunk.  For each (l, h),
+ * k_next[l][h] = the last (out_segments - chunk_segs) kept segments of the
+ * compressed cache (rows of k_comp, in order), followed by the Lq rows of the
+ * chunk's own k_cur; the same for v.  chunk_segs = Fc (frame mode) or Lq
+ * (token mode); out_segments counts segments of the result, so the next
+ * call's history is out_segments frames (frame mode: hist_frames =
+ * out_segments) or tokens, the older kept segments being dropped (a fixed
+ * window).  The compressed KV replaces the cache (Forcing-KV,
+ * "输出与工程收益") and the new chunk joins it; the window follows Deep
+ * Forcing's budget of 70-80% of a sliding window (section 5.1).
+ * k_next, v_next: [L][H][out_segments*seg_len][D]; they must not overlap the
+ * inputs.  A head that kept fewer than out_segments - chunk_segs segments gets
+ * zero rows there and FKV_ERR_DEVICE_ARG is recorded.  k_comp / v_comp may
+ * be NULL when out_segments == chunk_segs (chunk only); kept_cnt is always
+ * required.
+ * Denoising steps after the first reuse a chunk's selection and compressed
+ * cache by calling fkv_attend_compressed alone. */
+int32_t fkv_cache_advance(const fkv_params_t* p, const void* k_comp, const void* v_comp,
+                          const int32_t* kept_cnt, const void* k_cur, const void* v_cur,
+                          int64_t out_segments, void* k_next, void* v_next, void* ws,
+                          void* stream);
+
 /* Steps 1-5 in one call: score (dynamic / token heads), select, compact,
  * attend, all enqueued on `stream` in that order. */
 int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void* stream);

@@ -29,7 +29,7 @@ from ._lib import Params, StepIO
 __all__ = [
     "FkvError", "Params", "make_params", "params_for", "sizes", "allocate", "score_segments",
     "select_topk", "compact_gather", "attend_compressed", "step", "read_status", "library",
-    "step_launches", "make_step_io", "score_segments_noalloc",
+    "step_launches", "make_step_io", "score_segments_noalloc", "cache_advance",
 ]
 
 
@@ -227,6 +227,25 @@ def attend_compressed(p: Params, q_cur, k_cur, v_cur, k_comp, v_comp, kept_cnt, 
         _ptr(v_comp, "v_comp", dt, n["comp"]), _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]),
         _ptr(out, "out", dt, n["act_cur"]), _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
     _check(st, "fkv_attend_compressed")
+
+
+def cache_advance(p: Params, k_comp, v_comp, kept_cnt, k_cur, v_cur, out_segments: int, k_next,
+                  v_next, ws, stream=None):
+    """Next history cache (fkv_cache_advance): the last out_segments - chunk
+    kept segments of the compressed cache, then the chunk's own K/V."""
+    n, dt = _shapes(p), _act_dtype(p)
+    seg_len = p.frame_tokens if p.granularity == _lib.FKV_GRAN_FRAME else 1
+    out_n = p.num_layers * p.num_heads * out_segments * seg_len * p.head_dim
+    chunk_segs = (p.chunk_frames * p.frame_tokens) // seg_len
+    old = out_segments > chunk_segs
+    st = _lib.load().fkv_cache_advance(
+        ctypes.byref(p), _ptr(k_comp, "k_comp", dt, n["comp"], optional=not old),
+        _ptr(v_comp, "v_comp", dt, n["comp"], optional=not old),
+        _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]),
+        _ptr(k_cur, "k_cur", dt, n["act_cur"]), _ptr(v_cur, "v_cur", dt, n["act_cur"]),
+        int(out_segments), _ptr(k_next, "k_next", dt, out_n), _ptr(v_next, "v_next", dt, out_n),
+        _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
+    _check(st, "fkv_cache_advance")
 
 
 def make_step_io(p: Params, inputs: Dict[str, torch.Tensor], outputs: Dict[str, torch.Tensor]) -> StepIO:

@@ -330,6 +330,30 @@ int32_t fkv_attend_compressed(const fkv_params_t* p, const void* q_cur, const vo
                    static_cast<cudaStream_t>(stream));
 }
 
+int32_t fkv_cache_advance(const fkv_params_t* p, const void* k_comp, const void* v_comp,
+                          const int32_t* kept_cnt, const void* k_cur, const void* v_cur,
+                          int64_t out_segments, void* k_next, void* v_next, void* ws,
+                          void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  const int64_t chunk_segs = d.Lq / d.seg_len;
+  if (out_segments < chunk_segs || out_segments > d.max_kept + chunk_segs ||
+      out_segments * d.seg_len > kMaxRowsPerHead)
+    return FKV_ERR_SHAPE;
+  const bool old = out_segments > chunk_segs;
+  if ((old && (!k_comp || !v_comp)) || !kept_cnt || !k_cur || !v_cur || !k_next || !v_next)
+    return FKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {k_cur, v_cur, k_next, v_next};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FKV_ERR_INVALID_ARG;
+  if (old && (!aligned16(k_comp) || !aligned16(v_comp))) return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  return cuda_status(launch_advance(d, out_segments, k_comp, v_comp, kept_cnt, k_cur, v_cur,
+                                    k_next, v_next, status_ptr(ws),
+                                    static_cast<cudaStream_t>(stream)));
+}
+
 int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void* stream) {
   Dims d;
   int32_t st = make_dims(p, &d);

@@ -90,6 +90,10 @@ cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_
                                 const void* v_cur, const void* k_comp, const void* v_comp,
                                 const int32_t* kept_cnt, void* out, int32_t* status,
                                 cudaStream_t s);
+cudaError_t launch_advance(const Dims& d, int64_t out_segments, const void* k_comp,
+                           const void* v_comp, const int32_t* kept_cnt, const void* k_cur,
+                           const void* v_cur, void* k_next, void* v_next, int32_t* status,
+                           cudaStream_t s);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
 cudaError_t launch_attend_simt(const Dims& d, const void* q_cur, const void* k_cur,
                                const void* v_cur, const void* k_comp, const void* v_comp,

@@ -91,4 +91,82 @@ cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
   return cudaGetLastError();
 }
 
+// Next history cache: rows [0, keep*seg_len) of the output are the last
+// `keep` kept segments of the compressed cache, rows after them the chunk's
+// own rows.  grid = (blocks, L*H); same 16-byte streaming copy as above.
+__global__ void __launch_bounds__(kGatherThreads)
+advance_kernel(int32_t seg_len, int32_t max_kept, int32_t comp_rows, int32_t keep,
+               int32_t chunk_rows, int32_t vec_per_row, const uint4* __restrict__ k_comp,
+               const uint4* __restrict__ v_comp, const int32_t* __restrict__ kept_cnt,
+               const uint4* __restrict__ k_cur, const uint4* __restrict__ v_cur,
+               uint4* __restrict__ k_next, uint4* __restrict__ v_next, int32_t* status) {
+  const int lh = blockIdx.y;
+  int32_t cnt = kept_cnt[lh];
+  bool bad = cnt < keep || cnt > max_kept || int64_t(cnt) * seg_len > comp_rows;
+  if (bad && blockIdx.x == 0 && threadIdx.x == 0) report(status, FKV_ERR_DEVICE_ARG, lh);
+  const int64_t old_rows = int64_t(keep) * seg_len;
+  const int64_t out_rows = old_rows + chunk_rows;
+  const int64_t nvec = out_rows * vec_per_row;
+  const int64_t src0 = bad ? 0 : (int64_t(cnt) - keep) * seg_len;  // first kept row copied
+  const uint4* kc = k_comp + int64_t(lh) * comp_rows * vec_per_row;
+  const uint4* vc = v_comp + int64_t(lh) * comp_rows * vec_per_row;
+  const uint4* kn = k_cur + int64_t(lh) * chunk_rows * vec_per_row;
+  const uint4* vn = v_cur + int64_t(lh) * chunk_rows * vec_per_row;
+  uint4* kd = k_next + int64_t(lh) * out_rows * vec_per_row;
+  uint4* vd = v_next + int64_t(lh) * out_rows * vec_per_row;
+  const int64_t step = int64_t(gridDim.x) * kGatherThreads * kGatherUnroll;
+  for (int64_t base = int64_t(blockIdx.x) * kGatherThreads * kGatherUnroll + threadIdx.x;
+       base < nvec; base += step) {
+    uint4 kv[kGatherUnroll], vv[kGatherUnroll];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const int64_t i = base + int64_t(u) * kGatherThreads;
+      if (i < nvec) {
+        const int64_t r = i / vec_per_row, v = i - r * vec_per_row;
+        if (r < old_rows) {
+          if (bad) {  // not enough kept segments: leave zeros, error recorded
+            kv[u] = vv[u] = make_uint4(0, 0, 0, 0);
+          } else {
+            kv[u] = __ldcs(kc + (src0 + r) * vec_per_row + v);
+            vv[u] = __ldcs(vc + (src0 + r) * vec_per_row + v);
+          }
+        } else {
+          kv[u] = __ldcs(kn + (r - old_rows) * vec_per_row + v);
+          vv[u] = __ldcs(vn + (r - old_rows) * vec_per_row + v);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const int64_t i = base + int64_t(u) * kGatherThreads;
+      if (i < nvec) {
+        __stcs(kd + i, kv[u]);
+        __stcs(vd + i, vv[u]);
+      }
+    }
+  }
+}
+
+cudaError_t launch_advance(const Dims& d, int64_t out_segments, const void* k_comp,
+                           const void* v_comp, const int32_t* kept_cnt, const void* k_cur,
+                           const void* v_cur, void* k_next, void* v_next, int32_t* status,
+                           cudaStream_t s) {
+  const int vec_per_row = d.D * d.elem / 16;
+  const int64_t chunk_segs = d.Lq / d.seg_len;
+  const int64_t keep = out_segments - chunk_segs;
+  const int64_t out_rows = out_segments * d.seg_len;
+  const int64_t per_block = int64_t(kGatherThreads) * kGatherUnroll;
+  int64_t bx = (out_rows * vec_per_row + per_block - 1) / per_block;
+  if (bx < 1) bx = 1;
+  if (bx > 65535) bx = 65535;
+  dim3 grid(unsigned(bx), unsigned(d.LH));
+  advance_kernel<<<grid, kGatherThreads, 0, s>>>(
+      int32_t(d.seg_len), int32_t(d.max_kept), int32_t(d.comp_rows), int32_t(keep),
+      int32_t(d.Lq), vec_per_row, static_cast<const uint4*>(k_comp),
+      static_cast<const uint4*>(v_comp), kept_cnt, static_cast<const uint4*>(k_cur),
+      static_cast<const uint4*>(v_cur), static_cast<uint4*>(k_next), static_cast<uint4*>(v_next),
+      status);
+  return cudaGetLastError();
+}
+
 }  // namespace fkv

@@ -128,6 +128,26 @@ def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float)
     return out
 
 
+def advance(comp: np.ndarray, kept_count: int, seg_len: int, chunk: np.ndarray,
+            out_segments: int) -> np.ndarray:
+    """The next history cache of one head: the most recent kept segments of the
+    compressed cache followed by the chunk's own keys (or values).
+
+    Forcing-KV, "输出与工程收益": the compressed KV replaces the original cache;
+    the chunk just generated joins the history for the next chunk
+    ("输入与整体流程": history KV grows frame by frame); a window keeps the
+    cache bounded (Deep Forcing, section 5.1: a budget of 70-80% of the
+    sliding window).  out_segments counts segments (frames, or tokens) of the
+    result, chunk segments included; the oldest kept segments are dropped.
+    comp [>= kept_count*seg_len][D], chunk [chunk_rows][D].
+    """
+    chunk_segs = chunk.shape[0] // seg_len
+    keep = out_segments - chunk_segs
+    assert 0 <= keep <= kept_count
+    old = comp[(kept_count - keep) * seg_len:kept_count * seg_len]
+    return np.concatenate([old, chunk], axis=0)
+
+
 def head_keep(*, granularity: str, dynamic: bool, mask_row, k: int, q_cur, k_hist,
               T: int, scale: float, score_stride: int = 1, q_score=None,
               sink: int = 0, recent: int = 0):
@@ -185,5 +205,5 @@ def kept_rows(kept: np.ndarray, granularity: str, T: int) -> int:
 
 __all__: List[str] = [
     "static_keep", "scoring_queries", "segment_mass", "top_k", "participative_phi",
-    "token_keep", "compact", "attention", "head_keep", "step", "kept_rows",
+    "token_keep", "compact", "attention", "advance", "head_keep", "step", "kept_rows",
 ]

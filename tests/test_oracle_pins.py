@@ -298,3 +298,17 @@ def test_token_step_scores_the_candidate_rows():
 def test_empty_history_keeps_nothing():
     assert orc.segment_mass(np.ones((2, 4)), np.zeros((0, 4)), 3, 0.5).shape == (0,)
     assert orc.top_k(np.zeros(0), 0).tolist() == []
+
+
+def test_advance_keeps_the_most_recent_segments_then_the_chunk():
+    T, D = 2, 3
+    comp = np.repeat(np.arange(10, dtype=np.float64)[:, None], D, axis=1)  # 5 kept frames
+    chunk = np.repeat(np.arange(100, 104, dtype=np.float64)[:, None], D, axis=1)  # 2 frames
+    got = orc.advance(comp, 5, T, chunk, out_segments=5)   # keep 3 kept frames + 2 chunk
+    assert got[:, 0].tolist() == [4, 5, 6, 7, 8, 9, 100, 101, 102, 103]
+    got = orc.advance(comp, 5, T, chunk, out_segments=2)   # chunk only
+    assert got[:, 0].tolist() == [100, 101, 102, 103]
+    got = orc.advance(comp, 4, 1, chunk[:1], out_segments=3)  # token mode: last 2 of 4 kept
+    assert got[:, 2].tolist() == [2, 3, 100]
+    with pytest.raises(AssertionError):
+        orc.advance(comp, 2, T, chunk, out_segments=6)

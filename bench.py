@@ -245,7 +245,7 @@ def run_ours(args, rank, world, local_rank):
         e = kev[i]
         e[0].record(stream)
         fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
-                           outs["seg_score"], outs["ws"])
+                           outs["seg_score"], outs["ws"], k_cur=x["k_cur"])
         e[1].record(stream)
         fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
                         x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])

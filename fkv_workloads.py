@@ -73,6 +73,7 @@ class Workload:
     recent_tokens: int = 0
     keep_tokens: int = 0  # C in the participative variant
     style: str = "video"  # "video" or "tiny"
+    score_with_chunk: bool = False  # chunk keys in the scoring normaliser
 
     @property
     def N(self) -> int:

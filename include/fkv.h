@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define FKV_ABI_VERSION 1
+#define FKV_ABI_VERSION 2
 
 typedef enum fkv_status {
   FKV_OK = 0,
@@ -71,6 +71,14 @@ typedef enum fkv_dtype { FKV_DTYPE_BF16 = 0, FKV_DTYPE_FP32 = 1 } fkv_dtype_t;
 /* Segment = one latent frame of T tokens (Forcing-KV), or one token (the
  * participative variant, where every head is dynamic). */
 typedef enum fkv_granularity { FKV_GRAN_FRAME = 0, FKV_GRAN_TOKEN = 1 } fkv_granularity_t;
+
+/* fkv_params_t.flags bits. */
+#define FKV_FLAG_SCORE_WITH_CHUNK 1 /* frame mode: the scoring softmax of each
+                                       query row is normalised over the history
+                                       keys AND the chunk's own keys (the
+                                       attention the chunk computes); masses are
+                                       still per history frame.  Default (0):
+                                       history keys only. */
 
 typedef struct fkv_params {
   int32_t num_layers;    /* L >= 1: layers batched in one call (independent)  */
@@ -90,6 +98,7 @@ typedef struct fkv_params {
                             1/sqrt(D)                                          */
   int32_t dtype;         /* fkv_dtype_t                                        */
   int32_t granularity;   /* fkv_granularity_t                                  */
+  int32_t flags;         /* FKV_FLAG_* bits, 0 for the defaults                */
 } fkv_params_t;
 
 /* All inputs and outputs of fkv_step (device pointers, caller-owned). */
@@ -165,14 +174,15 @@ int32_t fkv_read_status(const void* ws, void* stream, int32_t* device_status, in
 /* Step 2: segment scores.
  * Frame mode (dynamic heads only; static rows of seg_score are written 0):
  *   seg_score[l][h][f] = sum_i sum_{j in frame f} softmax_j(scale * q_i . k_j),
- *   q_i = q_cur[l][h][i*score_stride], softmax over the N history keys.
- *   q_score is unused (may be NULL).
+ *   q_i = q_cur[l][h][i*score_stride], softmax over the N history keys (and
+ *   the Lq rows of k_cur too with FKV_FLAG_SCORE_WITH_CHUNK; k_cur is unused
+ *   and may be NULL otherwise).  q_score is unused (may be NULL).
  * Token mode (every head): seg_score[l][h][c] = sum_r q_score[l][h][r] .
  *   k_hist[l][h][S + c] for the candidates c = 0 .. N-S-R-1 (no scale).
  * Scores are float32.  Uses the scoring scratch of `ws`. */
 int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void* q_score,
-                           const void* k_hist, const uint8_t* head_role, float* seg_score,
-                           void* ws, void* stream);
+                           const void* k_hist, const void* k_cur, const uint8_t* head_role,
+                           float* seg_score, void* ws, void* stream);
 
 /* fkv_score_segments without a workspace argument, for callers that cannot
  * allocate device memory (e.g. a plugin that a host runtime hands only its
@@ -196,8 +206,8 @@ int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void*
  *  - Device-side errors of this call are not reported (there is no workspace
  *    status word for the caller to read). */
 int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void* q_cur, const void* q_score,
-                                   const void* k_hist, const uint8_t* head_role, float* seg_score,
-                                   void* stream);
+                                   const void* k_hist, const void* k_cur,
+                                   const uint8_t* head_role, float* seg_score, void* stream);
 
 /* Steps 1 and 3: kept segment lists.
  * Frame mode: static heads keep the frames with static_mask == 1; dynamic

@@ -52,9 +52,9 @@ def _check(status: int, where: str):
 def make_params(*, L: int, H: int, D: int, T: int, F: int, Fc: int, dtype: str = "bf16",
                 granularity: str = "frame", score_stride: int = 1, n_score_q: int = 0,
                 sink_tokens: int = 0, recent_tokens: int = 0, comp_rows: Optional[int] = None,
-                scale: Optional[float] = None) -> Params:
+                scale: Optional[float] = None, score_with_chunk: bool = False) -> Params:
     """fkv_params_t from keyword sizes.  comp_rows defaults to the worst case
-    (every history row kept)."""
+    (every history row kept).  score_with_chunk sets FKV_FLAG_SCORE_WITH_CHUNK."""
     p = Params()
     p.num_layers, p.num_heads, p.head_dim = L, H, D
     p.frame_tokens, p.hist_frames, p.chunk_frames = T, F, Fc
@@ -64,6 +64,7 @@ def make_params(*, L: int, H: int, D: int, T: int, F: int, Fc: int, dtype: str =
     p.scale = 1.0 / math.sqrt(D) if scale is None else scale
     p.dtype = {"bf16": _lib.FKV_DTYPE_BF16, "fp32": _lib.FKV_DTYPE_FP32}[dtype]
     p.granularity = {"frame": _lib.FKV_GRAN_FRAME, "token": _lib.FKV_GRAN_TOKEN}[granularity]
+    p.flags = _lib.FKV_FLAG_SCORE_WITH_CHUNK if score_with_chunk else 0
     return p
 
 
@@ -79,7 +80,8 @@ def params_for(w, comp_rows: Optional[int] = None) -> Params:
     return make_params(L=w.L, H=w.H, D=w.D, T=w.T, F=w.F, Fc=w.Fc, dtype=w.dtype,
                        granularity=w.granularity, score_stride=w.score_stride,
                        n_score_q=w.n_score_q, sink_tokens=w.sink_tokens,
-                       recent_tokens=w.recent_tokens, comp_rows=comp_rows, scale=w.scale)
+                       recent_tokens=w.recent_tokens, comp_rows=comp_rows, scale=w.scale,
+                       score_with_chunk=getattr(w, "score_with_chunk", False))
 
 
 def sizes(p: Params) -> Dict[str, int]:
@@ -165,20 +167,24 @@ def allocate(p: Params, device="cuda") -> Dict[str, torch.Tensor]:
     return out
 
 
-def score_segments(p: Params, q_cur, q_score, k_hist, head_role, seg_score, ws, stream=None):
+def score_segments(p: Params, q_cur, q_score, k_hist, head_role, seg_score, ws, stream=None,
+                   k_cur=None):
+    """Segment scores; k_cur (the chunk's keys) is needed with score_with_chunk."""
     n, dt = _shapes(p), _act_dtype(p)
     token = p.granularity == _lib.FKV_GRAN_TOKEN
     st = _lib.load().fkv_score_segments(
         ctypes.byref(p), _ptr(q_cur, "q_cur", dt, n["act_cur"], optional=token),
         _ptr(q_score, "q_score", dt, n["q_score"], optional=not token),
         _ptr(k_hist, "k_hist", dt, n["act_hist"]),
+        _ptr(k_cur, "k_cur", dt, n["act_cur"], optional=not (p.flags & _lib.FKV_FLAG_SCORE_WITH_CHUNK)),
         _ptr(head_role, "head_role", torch.uint8, n["heads"], optional=token),
         _ptr(seg_score, "seg_score", torch.float32, n["seg"]),
         _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
     _check(st, "fkv_score_segments")
 
 
-def score_segments_noalloc(p: Params, q_cur, q_score, k_hist, head_role, seg_score, stream=None):
+def score_segments_noalloc(p: Params, q_cur, q_score, k_hist, head_role, seg_score, stream=None,
+                           k_cur=None):
     """score_segments without a workspace: for callers that cannot allocate
     device memory.  The library's own static 4 MiB device scratch is used, so
     sizes needing more are rejected, and calls must not overlap on the GPU."""
@@ -188,6 +194,7 @@ def score_segments_noalloc(p: Params, q_cur, q_score, k_hist, head_role, seg_sco
         ctypes.byref(p), _ptr(q_cur, "q_cur", dt, n["act_cur"], optional=token),
         _ptr(q_score, "q_score", dt, n["q_score"], optional=not token),
         _ptr(k_hist, "k_hist", dt, n["act_hist"]),
+        _ptr(k_cur, "k_cur", dt, n["act_cur"], optional=not (p.flags & _lib.FKV_FLAG_SCORE_WITH_CHUNK)),
         _ptr(head_role, "head_role", torch.uint8, n["heads"], optional=token),
         _ptr(seg_score, "seg_score", torch.float32, n["seg"]), _stream(stream))
     _check(st, "fkv_score_segments_noalloc")

@@ -20,6 +20,7 @@ FKV_DTYPE_BF16 = 0
 FKV_DTYPE_FP32 = 1
 FKV_GRAN_FRAME = 0
 FKV_GRAN_TOKEN = 1
+FKV_FLAG_SCORE_WITH_CHUNK = 1
 
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -32,7 +33,7 @@ class Params(ctypes.Structure):
         ("frame_tokens", c_i32), ("hist_frames", c_i32), ("chunk_frames", c_i32),
         ("score_stride", c_i32), ("n_score_q", c_i32), ("sink_tokens", c_i32),
         ("recent_tokens", c_i32), ("comp_rows", c_i32), ("scale", c_f32),
-        ("dtype", c_i32), ("granularity", c_i32),
+        ("dtype", c_i32), ("granularity", c_i32), ("flags", c_i32),
     ]
 
 
@@ -61,8 +62,8 @@ SIGNATURES = {
     "fkv_exp2_emulated": (c_i32, [c_vp, c_vp, c_i64, c_vp]),
     "fkv_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
     "fkv_read_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
-    "fkv_score_segments": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
-    "fkv_score_segments_noalloc": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "fkv_score_segments": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "fkv_score_segments_noalloc": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "fkv_select_topk": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "fkv_compact_gather": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "fkv_attend_compressed": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),

@@ -17,7 +17,8 @@ WsLayout ws_layout(const Dims& d) {
   w.part_ml = w.row_ml = w.qbar = off;
   if (!d.token) {
     w.part_ml = off;
-    off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(d.F) * kScoreSplit * size_t(d.n_s));
+    off = align256(off + sizeof(float2) * size_t(d.LH) * (size_t(d.F) * kScoreSplit + 1) *
+                             size_t(d.n_s));
     w.row_ml = off;
     off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(d.n_s));
   } else {
@@ -57,6 +58,9 @@ static int32_t make_dims(const fkv_params_t* p, Dims* d) {
     return FKV_ERR_SHAPE;
   d->bf16 = p->dtype == FKV_DTYPE_BF16;
   d->token = p->granularity == FKV_GRAN_TOKEN;
+  if (p->flags & ~int32_t(FKV_FLAG_SCORE_WITH_CHUNK)) return FKV_ERR_INVALID_ARG;
+  d->score_with_chunk = (p->flags & FKV_FLAG_SCORE_WITH_CHUNK) != 0;
+  if (d->token && d->score_with_chunk) return FKV_ERR_UNSUPPORTED;  // phi has no softmax
   d->elem = d->bf16 ? 2 : 4;
   if (d->bf16) {
     if (d->D != 128) return FKV_ERR_UNSUPPORTED;
@@ -111,7 +115,8 @@ static char* ws_at(void* ws, size_t off) { return reinterpret_cast<char*>(ws) + 
 // ---- the five steps, after validation -------------------------------------
 
 static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, const void* k_hist,
-                        const uint8_t* head_role, float* seg_score, void* ws, cudaStream_t s) {
+                        const void* k_cur, const uint8_t* head_role, float* seg_score, void* ws,
+                        cudaStream_t s) {
   WsLayout w = ws_layout(d);
   if (d.token) {
     if (d.nseg == 0) return FKV_OK;
@@ -123,9 +128,9 @@ static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, c
   float2* part = reinterpret_cast<float2*>(ws_at(ws, w.part_ml));
   float2* rows = reinterpret_cast<float2*>(ws_at(ws, w.row_ml));
   // bf16: tensor-core scoring; fp32: CUDA-core scoring (fp32 accuracy mode).
-  cudaError_t e = d.bf16 ? launch_score_frame_sm100(d, q_cur, k_hist, head_role, part,
+  cudaError_t e = d.bf16 ? launch_score_frame_sm100(d, q_cur, k_hist, k_cur, head_role, part,
                                                     status_ptr(ws), s)
-                         : launch_score_frame_simt(d, q_cur, k_hist, head_role, part, s);
+                         : launch_score_frame_simt(d, q_cur, k_hist, k_cur, head_role, part, s);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(
       launch_score_frame_finalize(d, d.bf16 ? kScoreSplit : 1, head_role, part, rows, seg_score, s));
@@ -265,8 +270,8 @@ int32_t fkv_read_status(const void* ws, void* stream, int32_t* device_status, in
 }
 
 int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void* q_score,
-                           const void* k_hist, const uint8_t* head_role, float* seg_score,
-                           void* ws, void* stream) {
+                           const void* k_hist, const void* k_cur, const uint8_t* head_role,
+                           float* seg_score, void* ws, void* stream) {
   Dims d;
   int32_t st = make_dims(p, &d);
   if (st != FKV_OK) return st;
@@ -279,8 +284,9 @@ int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void*
     if (!aligned16(q_cur)) return FKV_ERR_INVALID_ARG;
   }
   if (!aligned16(k_hist)) return FKV_ERR_INVALID_ARG;
+  if (d.score_with_chunk && (!k_cur || !aligned16(k_cur))) return FKV_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws)) != FKV_OK) return st;
-  return do_score(d, q_cur, q_score, k_hist, head_role, seg_score, ws,
+  return do_score(d, q_cur, q_score, k_hist, k_cur, head_role, seg_score, ws,
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -372,7 +378,8 @@ int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void*
   if (d.token && !aligned16(io->q_score)) return FKV_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws)) != FKV_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = do_score(d, io->q_cur, io->q_score, io->k_hist, io->head_role, io->seg_score, ws, s)))
+  if ((st = do_score(d, io->q_cur, io->q_score, io->k_hist, io->k_cur, io->head_role,
+                     io->seg_score, ws, s)))
     return st;
   if ((st = do_select(d, io->seg_score, io->head_role, io->static_mask, io->k_per_head,
                       io->kept_idx, io->kept_cnt, ws, s)))

@@ -26,6 +26,7 @@ struct Dims {
   float scale;
   bool bf16;
   bool token;
+  bool score_with_chunk;  // frame mode: chunk keys in the scoring normaliser
   int elem;          // bytes per activation element
 };
 
@@ -36,7 +37,8 @@ constexpr int kScoreSplit = 2;
 // Workspace layout (byte offsets from the workspace base, 256-B aligned).
 struct WsLayout {
   size_t status;     // int32[2]: first device error, detail
-  size_t part_ml;    // frame mode: float2 [LH][F*kScoreSplit][n_s] per-sub-segment (max, sum)
+  size_t part_ml;    // frame mode: float2 [LH][F*kScoreSplit + 1][n_s] per-sub-segment
+                     // (max, sum); the last entry is the chunk's own keys
   size_t row_ml;     // frame mode: float2 [LH][n_s] per-row (max, sum)
   size_t qbar;       // token mode: float [LH][D] summed scoring queries
   size_t total;
@@ -67,7 +69,10 @@ __device__ __forceinline__ uint32_t ordered_key(float x) {
 
 // ---- launchers (each returns cudaGetLastError() of its launches) ----------
 cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
-                                    const uint8_t* head_role, float2* part_ml, cudaStream_t s);
+                                    const void* k_cur, const uint8_t* head_role, float2* part_ml,
+                                    cudaStream_t s);
+// part_ml holds, per head, F*split sub-segment entries followed (when
+// d.score_with_chunk) by one entry for the chunk's keys, each n_s rows.
 cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
                                         const float2* part_ml, float2* row_ml, float* seg_score,
                                         cudaStream_t s);
@@ -84,8 +89,8 @@ cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
                           const int32_t* kept_idx, const int32_t* kept_cnt, void* k_comp,
                           void* v_comp, int32_t* status, cudaStream_t s);
 cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const void* k_hist,
-                                     const uint8_t* head_role, float2* part_ml, int32_t* status,
-                                     cudaStream_t s);
+                                     const void* k_cur, const uint8_t* head_role, float2* part_ml,
+                                     int32_t* status, cudaStream_t s);
 cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_cur,
                                 const void* v_cur, const void* k_comp, const void* v_comp,
                                 const int32_t* kept_cnt, void* out, int32_t* status,

@@ -65,8 +65,8 @@ void* scratch_address(int32_t* st) {
 
 extern "C" int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void* q_cur,
                                               const void* q_score, const void* k_hist,
-                                              const uint8_t* head_role, float* seg_score,
-                                              void* stream) {
+                                              const void* k_cur, const uint8_t* head_role,
+                                              float* seg_score, void* stream) {
   int32_t st = fkv_check_params(p);
   if (st != FKV_OK) return st;
   size_t need = 0;
@@ -91,5 +91,6 @@ extern "C" int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void*
   }
   // Same validation and kernels as fkv_score_segments, with the static array
   // (256-byte aligned, large enough as checked above) as the workspace.
-  return fkv_score_segments(p, q_cur, q_score, k_hist, head_role, seg_score, scratch, stream);
+  return fkv_score_segments(p, q_cur, q_score, k_hist, k_cur, head_role, seg_score, scratch,
+                            stream);
 }

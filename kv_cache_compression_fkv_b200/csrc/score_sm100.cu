@@ -49,7 +49,8 @@ struct ScoreBars {
 constexpr size_t kScoreSmem = kSOffBar + sizeof(ScoreBars) + 1024;
 
 struct ScoreArgs {
-  int T, G;  // tokens per frame; sub-segments per head (F * kScoreSplit)
+  int T, G, E;  // tokens per frame; history sub-segments (F * kScoreSplit); entries per head
+  int Lq, with_chunk;
   int64_t n_s;
   float sl2;
   const uint8_t* head_role;
@@ -77,14 +78,26 @@ __device__ __forceinline__ float2 merge_ml(float2 a, float2 b) {
 
 __global__ void __launch_bounds__(kScoreThreads, 2)
 score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
-                   const __grid_constant__ CUtensorMap tm_k, const ScoreArgs a) {
+                   const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_kc, const ScoreArgs a) {
   const int qt = blockIdx.x, g = blockIdx.y, lh = blockIdx.z;
   if (!a.head_role[lh]) return;  // static head: nothing to score (uniform per CTA)
-  const int f = g / kScoreSplit, sub = g - f * kScoreSplit;
-  const int nb = (a.T + 127) / 128;
-  const int nbh = (nb + 1) / 2;
-  const int b0 = sub ? nbh : 0, b1 = sub ? nb : nbh;
-  float2* out = a.part_ml + (int64_t(lh) * a.G + g) * a.n_s;
+  // Key range of this CTA: a history sub-segment, or (last entry) the chunk's
+  // own keys when they join the normaliser.
+  const bool chunk = g >= a.G;
+  const CUtensorMap* tmk = chunk ? &tm_kc : &tm_k;
+  int row0, nkeys;
+  if (chunk) {
+    row0 = 0;
+    nkeys = a.Lq;
+  } else {
+    const int f = g / kScoreSplit, sub = g - f * kScoreSplit;
+    const int nbh = ((a.T + 127) / 128 + 1) / 2;
+    row0 = f * a.T + (sub ? nbh * 128 : 0);
+    nkeys = sub ? a.T - nbh * 128 : (a.T < nbh * 128 ? a.T : nbh * 128);
+  }
+  const int b0 = 0, b1 = nkeys > 0 ? (nkeys + 127) / 128 : 0;
+  float2* out = a.part_ml + (int64_t(lh) * a.E + g) * a.n_s;
   if (b0 >= b1) {  // empty sub-segment (a frame of one block): neutral statistics
     const int64_t i = int64_t(qt) * 128 + threadIdx.x;
     if (threadIdx.x < 128 && i < a.n_s) out[i] = make_float2(-INFINITY, 0.f);
@@ -123,7 +136,7 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
   if (warp == kScoreProducerWarp) {
     if (lane == 0) {
       prefetch_tmap(&tm_qs);
-      prefetch_tmap(&tm_k);
+      prefetch_tmap(tmk);
       mbar_expect_tx(&bars->q_full, kTileBytes);
       tma_load_tile(sm + kSOffQ, &tm_qs, &bars->q_full, qt * 128, lh);
       uint32_t issued = 0;
@@ -131,7 +144,7 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
         const uint32_t s = issued % kScoreStages, u = issued / kScoreStages;
         if (!mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort)) break;
         mbar_expect_tx(&bars->k_full[s], kTileBytes);
-        tma_load_tile(sm + kSOffK + s * kTileBytes, &tm_k, &bars->k_full[s], f * a.T + b * 128, lh);
+        tma_load_tile(sm + kSOffK + s * kTileBytes, tmk, &bars->k_full[s], row0 + b * 128, lh);
       }
       for (uint32_t i = issued > kScoreStages ? issued - kScoreStages : 0; i < issued; ++i)
         drain_wait_s(&bars->k_full[i % kScoreStages], (i / kScoreStages) & 1);
@@ -164,7 +177,7 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
     bool ok = true;
     for (uint32_t it = 0; ok && it < uint32_t(b1 - b0); ++it) {
       const uint32_t sb = it & 1, su = it >> 1;
-      const int cols_left = a.T - (b0 + int(it)) * 128 - 64 * half;
+      const int cols_left = nkeys - int(it) * 128 - 64 * half;
       const int nv = cols_left < 0 ? 0 : (cols_left < 64 ? cols_left : 64);
       if (!(ok = warp_wait_s(&bars->s_full[sb], su & 1, abort))) break;
       tc_fence_after();
@@ -223,17 +236,25 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
 }  // namespace sm100
 
 cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const void* k_hist,
-                                     const uint8_t* head_role, float2* part_ml, int32_t* status,
-                                     cudaStream_t s) {
+                                     const void* k_cur, const uint8_t* head_role, float2* part_ml,
+                                     int32_t* status, cudaStream_t s) {
   using namespace sm100;
   const uint64_t row_b = 128 * 2;
-  CUtensorMap tqs, tk;
+  CUtensorMap tqs, tk, tkc;
   if (!make_tmap_bf16(&tqs, q_cur, d.n_s, d.LH, row_b * d.stride, d.Lq * row_b) ||
       !make_tmap_bf16(&tk, k_hist, d.N, d.LH, row_b, d.N * row_b))
     return cudaErrorInvalidValue;
+  if (d.score_with_chunk) {
+    if (!make_tmap_bf16(&tkc, k_cur, d.Lq, d.LH, row_b, d.Lq * row_b)) return cudaErrorInvalidValue;
+  } else {
+    tkc = tk;  // never read
+  }
   ScoreArgs a;
   a.T = d.T;
   a.G = d.F * kScoreSplit;
+  a.E = a.G + 1;
+  a.Lq = int(d.Lq);
+  a.with_chunk = d.score_with_chunk ? 1 : 0;
   a.n_s = d.n_s;
   a.sl2 = d.scale * 1.4426950408889634f;
   a.head_role = head_role;
@@ -242,8 +263,8 @@ cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const voi
   cudaError_t e = cudaFuncSetAttribute(score_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(kScoreSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid(unsigned((d.n_s + 127) / 128), unsigned(a.G), unsigned(d.LH));
-  score_sm100_kernel<<<grid, kScoreThreads, kScoreSmem, s>>>(tqs, tk, a);
+  dim3 grid(unsigned((d.n_s + 127) / 128), unsigned(a.G + a.with_chunk), unsigned(d.LH));
+  score_sm100_kernel<<<grid, kScoreThreads, kScoreSmem, s>>>(tqs, tk, tkc, a);
   return cudaGetLastError();
 }
 

@@ -60,7 +60,8 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t n_s, float sl2,
                            const T* __restrict__ q_cur, const T* __restrict__ k_hist,
-                           const uint8_t* __restrict__ head_role, float2* __restrict__ part_ml) {
+                           const T* __restrict__ k_cur, const uint8_t* __restrict__ head_role,
+                           float2* __restrict__ part_ml) {
   const int lh = blockIdx.z;
   if (!head_role[lh]) return;
   extern __shared__ float smem[];
@@ -72,9 +73,12 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
   load_tile(Qs, kBQ, q_cur + (int64_t(lh) * Lq + row0 * stride) * D, int64_t(stride) * D, nq, D);
   const int r = threadIdx.x >> 3, c8 = threadIdx.x & 7;
   float m = -INFINITY, l = 0.f;
-  const T* kf = k_hist + (int64_t(lh) * F * T_ + int64_t(f) * T_) * D;
-  for (int k0 = 0; k0 < T_; k0 += kBK) {
-    const int nk = min(kBK, T_ - k0);
+  // f < F: history frame f; f == F: the chunk's own keys (normaliser only).
+  const bool chunk = f == F;
+  const T* kf = chunk ? k_cur + int64_t(lh) * Lq * D : k_hist + (int64_t(lh) * F * T_ + int64_t(f) * T_) * D;
+  const int nkeys = chunk ? int(Lq) : T_;
+  for (int k0 = 0; k0 < nkeys; k0 += kBK) {
+    const int nk = min(kBK, nkeys - k0);
     __syncthreads();
     load_tile(Ks, kBK, kf + int64_t(k0) * D, D, nk, D);
     __syncthreads();
@@ -99,7 +103,7 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
     l = l * exp2f(m - mn) + ps;
     m = mn;
   }
-  if (c8 == 0 && r < nq) part_ml[(int64_t(lh) * F + f) * n_s + row0 + r] = make_float2(m, l);
+  if (c8 == 0 && r < nq) part_ml[(int64_t(lh) * (F + 1) + f) * n_s + row0 + r] = make_float2(m, l);
 }
 
 // Frame masses from the partial statistics of G = F*split sub-segments per
@@ -112,17 +116,18 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
 constexpr int kFinThreads = 1024;
 
 __global__ void __launch_bounds__(kFinThreads)
-score_finalize_kernel(int F, int split, int64_t n_s, const uint8_t* __restrict__ head_role,
-                      const float2* __restrict__ part_ml, float2* __restrict__ row_ml,
-                      float* __restrict__ seg_score) {
+score_finalize_kernel(int F, int split, int with_chunk, int64_t n_s,
+                      const uint8_t* __restrict__ head_role, const float2* __restrict__ part_ml,
+                      float2* __restrict__ row_ml, float* __restrict__ seg_score) {
   const int lh = blockIdx.x;
-  const int G = F * split;
+  const int G = F * split + with_chunk;  // entries in the row normaliser
+  const int E = F * split + 1;           // entries per head in part_ml
   float* out = seg_score + int64_t(lh) * F;
   if (!head_role[lh]) {
     for (int f = threadIdx.x; f < F; f += blockDim.x) out[f] = 0.f;
     return;
   }
-  const float2* p = part_ml + int64_t(lh) * G * n_s;
+  const float2* p = part_ml + int64_t(lh) * E * n_s;
   float2* rm = row_ml + int64_t(lh) * n_s;
   for (int64_t i = threadIdx.x; i < n_s; i += blockDim.x) {
     float M = -INFINITY;
@@ -157,26 +162,29 @@ score_finalize_kernel(int F, int split, int64_t n_s, const uint8_t* __restrict__
 }
 
 cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
-                                    const uint8_t* head_role, float2* part_ml, cudaStream_t s) {
+                                    const void* k_cur, const uint8_t* head_role, float2* part_ml,
+                                    cudaStream_t s) {
   const size_t smem = sizeof(float) * 2 * kBQ * kLd;
-  dim3 grid(unsigned((d.n_s + kBQ - 1) / kBQ), unsigned(d.F), unsigned(d.LH));
+  dim3 grid(unsigned((d.n_s + kBQ - 1) / kBQ), unsigned(d.F + (d.score_with_chunk ? 1 : 0)),
+            unsigned(d.LH));
   const float sl2 = d.scale * kLog2e;
   if (d.bf16)
     score_frame_partial_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
         d.D, d.T, d.F, d.Lq, d.stride, d.n_s, sl2, static_cast<const __nv_bfloat16*>(q_cur),
-        static_cast<const __nv_bfloat16*>(k_hist), head_role, part_ml);
+        static_cast<const __nv_bfloat16*>(k_hist), static_cast<const __nv_bfloat16*>(k_cur),
+        head_role, part_ml);
   else
     score_frame_partial_kernel<float><<<grid, kThreads, smem, s>>>(
         d.D, d.T, d.F, d.Lq, d.stride, d.n_s, sl2, static_cast<const float*>(q_cur),
-        static_cast<const float*>(k_hist), head_role, part_ml);
+        static_cast<const float*>(k_hist), static_cast<const float*>(k_cur), head_role, part_ml);
   return cudaGetLastError();
 }
 
 cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
                                         const float2* part_ml, float2* row_ml, float* seg_score,
                                         cudaStream_t s) {
-  score_finalize_kernel<<<d.LH, kFinThreads, 0, s>>>(d.F, split, d.n_s, head_role, part_ml,
-                                                     row_ml, seg_score);
+  score_finalize_kernel<<<d.LH, kFinThreads, 0, s>>>(d.F, split, d.score_with_chunk ? 1 : 0,
+                                                     d.n_s, head_role, part_ml, row_ml, seg_score);
   return cudaGetLastError();
 }
 

@@ -43,7 +43,8 @@ def scoring_queries(q_cur: np.ndarray, stride: int) -> np.ndarray:
     return q_cur[0::stride]
 
 
-def segment_mass(q_rows: np.ndarray, k_hist: np.ndarray, T: int, scale: float) -> np.ndarray:
+def segment_mass(q_rows: np.ndarray, k_hist: np.ndarray, T: int, scale: float,
+                 k_chunk: Optional[np.ndarray] = None) -> np.ndarray:
     """Per-frame softmax attention mass of a dynamic head.
 
     Forcing-KV, "关键模块" 3 (dynamic similarity pruning): the history cache is
@@ -51,21 +52,25 @@ def segment_mass(q_rows: np.ndarray, k_hist: np.ndarray, T: int, scale: float) -
     queries.  Read as: z_ij = scale * q_i . k_j over all N history keys,
     p_ij = exp(z_ij) / sum_j' exp(z_ij') (per query row, history keys only),
     mass_f = sum_i sum_{j in frame f} p_ij.
+    With k_chunk given, the normaliser of each row also runs over the chunk's
+    own keys (the attention the chunk actually computes); the masses are still
+    those of the history frames.
 
-    q_rows [n_s][D], k_hist [F*T][D] -> mass [F].
+    q_rows [n_s][D], k_hist [F*T][D], k_chunk [Lq][D] or None -> mass [F].
     """
     n_s = q_rows.shape[0]
     N = k_hist.shape[0]
     F = N // T
     if F == 0:  # empty history: nothing to score
         return np.zeros(0)
+    keys = k_hist if k_chunk is None else np.concatenate([k_hist, k_chunk], axis=0)
     per_row = np.empty((n_s, F), dtype=np.float64)
     for r0 in range(0, n_s, _ROW_BLOCK):
-        z = scale * (q_rows[r0:r0 + _ROW_BLOCK] @ k_hist.T)
+        z = scale * (q_rows[r0:r0 + _ROW_BLOCK] @ keys.T)
         z = z - z.max(axis=1, keepdims=True)
         e = np.exp(z)
         p = e / e.sum(axis=1, keepdims=True)
-        per_row[r0:r0 + _ROW_BLOCK] = p.reshape(p.shape[0], F, T).sum(axis=2)
+        per_row[r0:r0 + _ROW_BLOCK] = p[:, :N].reshape(p.shape[0], F, T).sum(axis=2)
     return per_row.sum(axis=0)
 
 
@@ -150,13 +155,14 @@ def advance(comp: np.ndarray, kept_count: int, seg_len: int, chunk: np.ndarray,
 
 def head_keep(*, granularity: str, dynamic: bool, mask_row, k: int, q_cur, k_hist,
               T: int, scale: float, score_stride: int = 1, q_score=None,
-              sink: int = 0, recent: int = 0):
-    """Selection for one (layer, head): (kept segment ids, segment scores or None)."""
+              sink: int = 0, recent: int = 0, k_chunk=None):
+    """Selection for one (layer, head): (kept segment ids, segment scores or None).
+    k_chunk: include the chunk's own keys in the scoring normaliser."""
     N = k_hist.shape[0]
     if granularity == "frame":
         if not dynamic:
             return static_keep(mask_row), None
-        mass = segment_mass(scoring_queries(q_cur, score_stride), k_hist, T, scale)
+        mass = segment_mass(scoring_queries(q_cur, score_stride), k_hist, T, scale, k_chunk)
         return top_k(mass, k), mass
     phi = participative_phi(q_score, k_hist[sink:N - recent])
     return token_keep(phi, N, sink, recent, k), phi

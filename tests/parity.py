@@ -107,7 +107,8 @@ def check_step(w, inputs_cpu, res, heads=None, rows=None, check_comp=True):
             k=k_sel, q_cur=q_cur, k_hist=k_hist,
             T=w.T, scale=w.scale, score_stride=w.score_stride,
             q_score=None if "q_score" not in inputs_cpu else x("q_score", l, h),
-            sink=w.sink_tokens, recent=w.recent_tokens)
+            sink=w.sink_tokens, recent=w.recent_tokens,
+            k_chunk=x("k_cur", l, h) if getattr(w, "score_with_chunk", False) else None)
         kept_g = gpu_kept(res, l, h)
         if score_o is not None and len(score_o) > 0:
             sg = res["seg_score"][l, h].numpy().astype(np.float64)

@@ -53,7 +53,7 @@ def test_struct_layout_matches_header(tmp_path, lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fkv_abi_version() == 1
+    assert lib.fkv_abi_version() == 2
     for code in range(8):
         assert lib.fkv_status_string(code).decode().startswith("FKV_")
     assert lib.fkv_status_string(99) == b"FKV_ERR_UNKNOWN"
@@ -88,13 +88,20 @@ def test_param_validation(lib):
     tok.sink_tokens = 180
     assert chk(tok) == _lib.FKV_ERR_SHAPE                       # S + R > N
     assert lib.fkv_check_params(None) == _lib.FKV_ERR_INVALID_ARG
+    p = _p()
+    p.flags = 4                                                  # unknown flag bit
+    assert chk(p) == _lib.FKV_ERR_INVALID_ARG
+    assert chk(_p(score_with_chunk=True)) == _lib.FKV_OK
+    assert chk(_p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8,
+                  score_with_chunk=True)) == _lib.FKV_ERR_UNSUPPORTED
 
 
 def test_derived_sizes(lib):
     s = fkv.sizes(_p())
     assert s["nseg"] == 6 and s["max_kept"] == 6 and s["max_comp_rows"] == 192
     # status block + (max, sum) per frame and scoring row + (max, sum) per row
-    assert s["ws_bytes"] == 256 + 4 * 6 * 2 * 32 * 8 + 4 * 32 * 8  # 2 sub-segments per frame
+    # 2 sub-segments per frame + the chunk entry, then per-row merges
+    assert s["ws_bytes"] == 256 + 4 * (6 * 2 + 1) * 32 * 8 + 4 * 32 * 8
     t = fkv.sizes(_p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8))
     assert t["nseg"] == 192 - 80 and t["max_kept"] == 192 and t["max_comp_rows"] == 192
 
@@ -102,9 +109,11 @@ def test_derived_sizes(lib):
 def test_null_and_misaligned_pointers_fail_before_launch(lib):
     p = _p()
     fake = 1 << 20  # never dereferenced: validation fails first
-    assert lib.fkv_score_segments(ctypes.byref(p), fake, None, None, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
-    assert lib.fkv_score_segments(ctypes.byref(p), fake + 8, None, fake, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
-    assert lib.fkv_score_segments(ctypes.byref(p), fake, None, fake, fake, fake, fake + 16, None) == _lib.FKV_ERR_WORKSPACE
+    assert lib.fkv_score_segments(ctypes.byref(p), fake, None, None, None, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_score_segments(ctypes.byref(p), fake + 8, None, fake, None, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_score_segments(ctypes.byref(p), fake, None, fake, None, fake, fake, fake + 16, None) == _lib.FKV_ERR_WORKSPACE
+    pc = _p(score_with_chunk=True)                                # needs k_cur
+    assert lib.fkv_score_segments(ctypes.byref(pc), fake, None, fake, None, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
     assert lib.fkv_select_topk(ctypes.byref(p), fake, None, fake, fake, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
     assert lib.fkv_compact_gather(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, None) == _lib.FKV_ERR_INVALID_ARG
     assert lib.fkv_attend_compressed(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, None, None) == _lib.FKV_ERR_WORKSPACE

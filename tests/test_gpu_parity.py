@@ -97,3 +97,26 @@ def test_480p_30_layers(cuda_device):
     heads = [(l, h) for l in (0, 11, 29) for h in range(w.H)]
     st = parity.check_step(w, x, res, rows=rows, heads=heads)
     print("30 layers", st)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_scoring_normalised_with_the_chunk(cuda_device, dtype):
+    """FKV_FLAG_SCORE_WITH_CHUNK: each scoring row's softmax also runs over the
+    chunk's own keys (ragged tiles everywhere: T = 200, Lq = 400)."""
+    w = wl.scaled(wl.get("480p"), name=f"chunknorm_{dtype}", H=4, T=200, F=7, Fc=2, n_static=2,
+                  static_frames=(0, 3, 6), k_dynamic=4, score_stride=3, dtype=dtype, seed=23,
+                  score_with_chunk=True)
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    st = parity.check_step(w, x, res)
+    assert st["score_rel"] <= parity.SCORE_REL
+
+
+def test_480p_scoring_normalised_with_the_chunk(cuda_device):
+    w = wl.scaled(wl.get("480p"), score_with_chunk=True)
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    rows = wl.sample_rows(w.Lq, 16, seed=8)
+    heads = [(0, h) for h in range(w.H) if x["head_role"][0, h]]
+    st = parity.check_step(w, x, res, rows=rows, heads=heads)
+    print("480p score_with_chunk", st)

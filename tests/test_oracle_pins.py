@@ -312,3 +312,22 @@ def test_advance_keeps_the_most_recent_segments_then_the_chunk():
     assert got[:, 2].tolist() == [2, 3, 100]
     with pytest.raises(AssertionError):
         orc.advance(comp, 2, T, chunk, out_segments=6)
+
+
+def test_mass_with_chunk_in_the_normaliser_closed_form():
+    """Frame keys c_f * u, chunk keys c_x * u (Lq of them): the normaliser of row
+    i gains Lq * exp(s a_i c_x); masses are still per history frame."""
+    a, c, cx, T, Lq, D, scale = [1.5, -0.8, 2.0], [0.3, -1.2, 2.5], 0.7, 4, 6, 8, 0.6
+    q, k = _closed_form_inputs(a, c, T, D, scale)
+    u = np.ones(D) / math.sqrt(D)
+    kc = np.tile(cx * u, (Lq, 1))
+    got = orc.segment_mass(q, k, T, scale, k_chunk=kc)
+    exp = []
+    for cf in c:
+        tot = 0.0
+        for ai in a:
+            den = T * sum(math.exp(scale * ai * cg) for cg in c) + Lq * math.exp(scale * ai * cx)
+            tot += T * math.exp(scale * ai * cf) / den
+        exp.append(tot)
+    np.testing.assert_allclose(got, exp, rtol=1e-13)
+    assert got.sum() < len(a)  # part of each row's mass now sits on the chunk

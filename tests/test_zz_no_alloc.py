@@ -27,7 +27,7 @@ def _noalloc(p, d, seg_score):
     ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
     return lib.fkv_score_segments_noalloc(
         ctypes.byref(p), ptr(d.get("q_cur")), ptr(d.get("q_score")), ptr(d["k_hist"]),
-        ptr(d.get("head_role")), seg_score.data_ptr(),
+        ptr(d.get("k_cur")), ptr(d.get("head_role")), seg_score.data_ptr(),
         torch.cuda.current_stream().cuda_stream)
 
 

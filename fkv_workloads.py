@@ -74,6 +74,9 @@ class Workload:
     keep_tokens: int = 0  # C in the participative variant
     style: str = "video"  # "video" or "tiny"
     score_with_chunk: bool = False  # chunk keys in the scoring normaliser
+    # static heads keep tokens: every token of frame 0 and the first and last
+    # T/8 tokens of each other history frame (a chunk-boundary-like pattern)
+    static_token_mask: bool = False
 
     @property
     def N(self) -> int:
@@ -187,12 +190,20 @@ def _layer(w: Workload, seed: int):
         out["v_hist"], out["v_cur"] = v_all[:, : F * T], v_all[:, F * T:]
         if w.granularity == "token":
             out["q_score"] = rng.standard_normal((H, w.n_score_q, D), dtype=np.float32)
-    mask = np.zeros((H, F), dtype=np.uint8)
+    mask = np.zeros((H, F * T if w.static_token_mask else F), dtype=np.uint8)
     kph = np.zeros(H, dtype=np.int32)
     if w.granularity == "frame":
+        edge = max(1, T // 8)
         for h in range(H):
             if role[h] == 0:
-                mask[h, list(w.static_frames)] = 1
+                if w.static_token_mask:
+                    tok = mask[h].reshape(F, T)
+                    tok[:, :edge] = 1
+                    tok[:, T - edge:] = 1
+                    if F > 0:
+                        tok[0] = 1
+                else:
+                    mask[h, list(w.static_frames)] = 1
             else:
                 kph[h] = w.k_dynamic
     else:
@@ -220,7 +231,8 @@ def generate(w: Workload, threads: Optional[int] = None) -> Dict[str, torch.Tens
         shapes["q_score"] = (L, H, w.n_score_q, D)
     res = {k: torch.empty(s, dtype=dt) for k, s in shapes.items()}
     res["head_role"] = torch.empty((L, H), dtype=torch.uint8)
-    res["static_mask"] = torch.empty((L, H, w.F), dtype=torch.uint8)
+    res["static_mask"] = torch.empty((L, H, w.F * w.T if w.static_token_mask else w.F),
+                                     dtype=torch.uint8)
     res["k_per_head"] = torch.empty((L, H), dtype=torch.int32)
 
     def one(l):

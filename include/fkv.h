@@ -79,6 +79,18 @@ typedef enum fkv_granularity { FKV_GRAN_FRAME = 0, FKV_GRAN_TOKEN = 1 } fkv_gran
                                        attention the chunk computes); masses are
                                        still per history frame.  Default (0):
                                        history keys only. */
+#define FKV_FLAG_STATIC_TOKEN_MASK 2 /* frame mode: static heads keep fixed TOKEN
+                                       positions (e.g. chunk-boundary tokens):
+                                       static_mask is [L][H][N], one byte per
+                                       history token; every head's kept list
+                                       then holds token ids (a dynamic head's
+                                       kept frames expanded to their T tokens,
+                                       ascending), kept_idx is [L][H][N],
+                                       kept_cnt counts tokens, and the
+                                       compressed cache, attention and
+                                       fkv_cache_advance work on tokens
+                                       (segment = 1 row).  seg_score stays
+                                       [L][H][F]. */
 
 typedef struct fkv_params {
   int32_t num_layers;    /* L >= 1: layers batched in one call (independent)  */

@@ -52,9 +52,11 @@ def _check(status: int, where: str):
 def make_params(*, L: int, H: int, D: int, T: int, F: int, Fc: int, dtype: str = "bf16",
                 granularity: str = "frame", score_stride: int = 1, n_score_q: int = 0,
                 sink_tokens: int = 0, recent_tokens: int = 0, comp_rows: Optional[int] = None,
-                scale: Optional[float] = None, score_with_chunk: bool = False) -> Params:
+                scale: Optional[float] = None, score_with_chunk: bool = False,
+                static_token_mask: bool = False) -> Params:
     """fkv_params_t from keyword sizes.  comp_rows defaults to the worst case
-    (every history row kept).  score_with_chunk sets FKV_FLAG_SCORE_WITH_CHUNK."""
+    (every history row kept).  score_with_chunk / static_token_mask set
+    FKV_FLAG_SCORE_WITH_CHUNK / FKV_FLAG_STATIC_TOKEN_MASK."""
     p = Params()
     p.num_layers, p.num_heads, p.head_dim = L, H, D
     p.frame_tokens, p.hist_frames, p.chunk_frames = T, F, Fc
@@ -64,7 +66,8 @@ def make_params(*, L: int, H: int, D: int, T: int, F: int, Fc: int, dtype: str =
     p.scale = 1.0 / math.sqrt(D) if scale is None else scale
     p.dtype = {"bf16": _lib.FKV_DTYPE_BF16, "fp32": _lib.FKV_DTYPE_FP32}[dtype]
     p.granularity = {"frame": _lib.FKV_GRAN_FRAME, "token": _lib.FKV_GRAN_TOKEN}[granularity]
-    p.flags = _lib.FKV_FLAG_SCORE_WITH_CHUNK if score_with_chunk else 0
+    p.flags = ((_lib.FKV_FLAG_SCORE_WITH_CHUNK if score_with_chunk else 0) |
+               (_lib.FKV_FLAG_STATIC_TOKEN_MASK if static_token_mask else 0))
     return p
 
 
@@ -72,8 +75,13 @@ def params_for(w, comp_rows: Optional[int] = None) -> Params:
     """Params of a workload description (an object with the fields of
     ``fkv_workloads.Workload``).  comp_rows defaults to the rows the budgets
     keep: max(static mask size, k) * T in frame mode, S + C + R in token mode."""
+    token_mask = getattr(w, "static_token_mask", False)
     if comp_rows is None:
-        if w.granularity == "frame":
+        if w.granularity == "frame" and token_mask:
+            edge = max(1, w.T // 8)
+            static_rows = (w.T + (w.F - 1) * 2 * edge) if w.F > 0 else 0
+            comp_rows = max(static_rows, w.k_dynamic * w.T)
+        elif w.granularity == "frame":
             comp_rows = max(len(w.static_frames), w.k_dynamic) * w.T
         else:
             comp_rows = w.sink_tokens + w.keep_tokens + w.recent_tokens
@@ -81,7 +89,8 @@ def params_for(w, comp_rows: Optional[int] = None) -> Params:
                        granularity=w.granularity, score_stride=w.score_stride,
                        n_score_q=w.n_score_q, sink_tokens=w.sink_tokens,
                        recent_tokens=w.recent_tokens, comp_rows=comp_rows, scale=w.scale,
-                       score_with_chunk=getattr(w, "score_with_chunk", False))
+                       score_with_chunk=getattr(w, "score_with_chunk", False),
+                       static_token_mask=token_mask)
 
 
 def sizes(p: Params) -> Dict[str, int]:
@@ -141,7 +150,9 @@ def _shapes(p: Params) -> Dict[str, int]:
     N = p.hist_frames * p.frame_tokens
     return {
         "act_cur": L * H * Lq * D, "act_hist": L * H * N * D, "q_score": L * H * p.n_score_q * D,
-        "heads": L * H, "mask": L * H * p.hist_frames, "seg": L * H * s["nseg"],
+        "heads": L * H,
+        "mask": L * H * (N if p.flags & _lib.FKV_FLAG_STATIC_TOKEN_MASK else p.hist_frames),
+        "seg": L * H * s["nseg"],
         "kept": L * H * s["max_kept"], "comp": L * H * p.comp_rows * D, "ws": s["ws_bytes"],
     }
 

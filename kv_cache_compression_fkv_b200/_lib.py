@@ -21,6 +21,7 @@ FKV_DTYPE_FP32 = 1
 FKV_GRAN_FRAME = 0
 FKV_GRAN_TOKEN = 1
 FKV_FLAG_SCORE_WITH_CHUNK = 1
+FKV_FLAG_STATIC_TOKEN_MASK = 2
 
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 

@@ -58,9 +58,12 @@ static int32_t make_dims(const fkv_params_t* p, Dims* d) {
     return FKV_ERR_SHAPE;
   d->bf16 = p->dtype == FKV_DTYPE_BF16;
   d->token = p->granularity == FKV_GRAN_TOKEN;
-  if (p->flags & ~int32_t(FKV_FLAG_SCORE_WITH_CHUNK)) return FKV_ERR_INVALID_ARG;
+  if (p->flags & ~int32_t(FKV_FLAG_SCORE_WITH_CHUNK | FKV_FLAG_STATIC_TOKEN_MASK))
+    return FKV_ERR_INVALID_ARG;
   d->score_with_chunk = (p->flags & FKV_FLAG_SCORE_WITH_CHUNK) != 0;
-  if (d->token && d->score_with_chunk) return FKV_ERR_UNSUPPORTED;  // phi has no softmax
+  d->static_token_mask = (p->flags & FKV_FLAG_STATIC_TOKEN_MASK) != 0;
+  if (d->token && (d->score_with_chunk || d->static_token_mask))
+    return FKV_ERR_UNSUPPORTED;  // frame-mode options
   d->elem = d->bf16 ? 2 : 4;
   if (d->bf16) {
     if (d->D != 128) return FKV_ERR_UNSUPPORTED;
@@ -79,8 +82,8 @@ static int32_t make_dims(const fkv_params_t* p, Dims* d) {
     d->stride = p->score_stride;
     d->n_s = (d->Lq + d->stride - 1) / d->stride;
     d->nseg = d->F;
-    d->max_kept = d->F;
-    d->seg_len = d->T;
+    d->max_kept = d->static_token_mask ? d->N : d->F;
+    d->seg_len = d->static_token_mask ? 1 : d->T;
   } else {
     if (p->sink_tokens < 0 || p->recent_tokens < 0) return FKV_ERR_SHAPE;
     d->S = p->sink_tokens;
@@ -142,6 +145,9 @@ static int32_t do_select(const Dims& d, const float* seg_score, const uint8_t* h
   if (d.token)
     return cuda_status(
         launch_select_token(d, seg_score, k_per_head, kept_idx, kept_cnt, status_ptr(ws), s));
+  if (d.static_token_mask)
+    return cuda_status(launch_select_frame_tokens(d, seg_score, head_role, static_mask, k_per_head,
+                                                  kept_idx, kept_cnt, status_ptr(ws), s));
   return cuda_status(launch_select_frame(d, seg_score, head_role, static_mask, k_per_head,
                                          kept_idx, kept_cnt, status_ptr(ws), s));
 }

@@ -27,6 +27,7 @@ struct Dims {
   bool bf16;
   bool token;
   bool score_with_chunk;  // frame mode: chunk keys in the scoring normaliser
+  bool static_token_mask; // frame mode: per-token static masks, kept lists in tokens
   int elem;          // bytes per activation element
 };
 
@@ -82,6 +83,10 @@ cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uin
                                 const uint8_t* static_mask, const int32_t* k_per_head,
                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                 cudaStream_t s);
+cudaError_t launch_select_frame_tokens(const Dims& d, const float* seg_score,
+                                       const uint8_t* head_role, const uint8_t* static_mask,
+                                       const int32_t* k_per_head, int32_t* kept_idx,
+                                       int32_t* kept_cnt, int32_t* status, cudaStream_t s);
 cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int32_t* k_per_head,
                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                 cudaStream_t s);

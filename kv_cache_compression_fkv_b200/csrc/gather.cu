@@ -84,7 +84,7 @@ cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
   if (bx > 65535) bx = 65535;
   dim3 grid(unsigned(bx), unsigned(d.LH));
   gather_kernel<<<grid, kGatherThreads, 0, s>>>(
-      int32_t(d.seg_len), int32_t(d.token ? d.N : d.F), int32_t(d.max_kept),
+      int32_t(d.seg_len), int32_t(d.seg_len == 1 ? d.N : d.F), int32_t(d.max_kept),
       int32_t(d.comp_rows), vec_per_row, d.N, static_cast<const uint4*>(k_hist),
       static_cast<const uint4*>(v_hist), kept_idx, kept_cnt, static_cast<uint4*>(k_comp),
       static_cast<uint4*>(v_comp), status);

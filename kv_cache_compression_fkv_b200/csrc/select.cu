@@ -204,6 +204,93 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
   }
 }
 
+// Frame mode with per-token static masks: kept lists in tokens.  Dynamic
+// heads rank their frames as above, then write the tokens of the kept frames
+// in order; static heads compact the ascending tokens of their mask (block
+// scan per 1024 tokens).  One 1024-thread CTA per (layer, head).
+__global__ void __launch_bounds__(kSelThreads)
+select_frame_tokens_kernel(int F, int T, int64_t N, const float* __restrict__ seg_score,
+                           const uint8_t* __restrict__ head_role,
+                           const uint8_t* __restrict__ static_mask,
+                           const int32_t* __restrict__ k_per_head, int32_t* __restrict__ kept_idx,
+                           int32_t* __restrict__ kept_cnt, int32_t* status) {
+  __shared__ uint32_t keys[1024];
+  __shared__ int32_t kf[1024];
+  __shared__ int warp_tot[kSelWarps];
+  __shared__ int s_cnt;
+  const int lh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* out = kept_idx + int64_t(lh) * N;
+  if (head_role[lh]) {
+    int k = k_per_head[lh];
+    if (k < 0 || k > F) {
+      if (tid == 0) report(status, FKV_ERR_DEVICE_ARG, lh);
+      k = k < 0 ? 0 : F;
+    }
+    uint32_t key = 0;
+    if (tid < F) keys[tid] = key = ordered_key(seg_score[int64_t(lh) * F + tid]);
+    __syncthreads();
+    bool keep = false;
+    if (tid < F) {
+      int rank = 0;
+      for (int g = 0; g < F; ++g) {
+        const uint32_t kg = keys[g];
+        rank += (kg > key) || (kg == key && g < tid);
+      }
+      keep = rank < k;
+    }
+    // ascending kept frames
+    const unsigned b = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) warp_tot[warp] = __popc(b);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      before += w < warp ? warp_tot[w] : 0;
+      total += warp_tot[w];
+    }
+    if (keep) kf[before + __popc(b & ((1u << lane) - 1u))] = tid;
+    __syncthreads();
+    const int64_t n_out = int64_t(total) * T;
+    for (int64_t o = tid; o < n_out; o += kSelThreads) {
+      const int64_t pfr = o / T;
+      out[o] = int32_t(int64_t(kf[pfr]) * T + (o - pfr * T));
+    }
+    if (tid == 0) kept_cnt[lh] = int32_t(n_out);
+    return;
+  }
+  // static head: tokens of the mask, ascending
+  const uint8_t* mk = static_mask + int64_t(lh) * N;
+  int64_t base = 0;
+  for (int64_t c0 = 0; c0 < N; c0 += kSelThreads) {
+    const int64_t j = c0 + tid;
+    const bool keep = j < N && mk[j] != 0;
+    const unsigned b = __ballot_sync(0xffffffffu, keep);
+    if (lane == 0) warp_tot[warp] = __popc(b);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < kSelWarps; ++w) {
+      before += w < warp ? warp_tot[w] : 0;
+      total += warp_tot[w];
+    }
+    __syncthreads();
+    if (keep) out[base + before + __popc(b & ((1u << lane) - 1u))] = int32_t(j);
+    base += total;
+  }
+  if (tid == 0) s_cnt = int(base);
+  __syncthreads();
+  if (tid == 0) kept_cnt[lh] = s_cnt;
+}
+
+cudaError_t launch_select_frame_tokens(const Dims& d, const float* seg_score,
+                                       const uint8_t* head_role, const uint8_t* static_mask,
+                                       const int32_t* k_per_head, int32_t* kept_idx,
+                                       int32_t* kept_cnt, int32_t* status, cudaStream_t s) {
+  select_frame_tokens_kernel<<<d.LH, kSelThreads, 0, s>>>(d.F, d.T, d.N, seg_score, head_role,
+                                                          static_mask, k_per_head, kept_idx,
+                                                          kept_cnt, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int32_t* k_per_head,
                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                 cudaStream_t s) {

@@ -38,6 +38,13 @@ def static_keep(mask_row: np.ndarray) -> np.ndarray:
     return np.flatnonzero(np.asarray(mask_row) != 0).astype(np.int64)
 
 
+def frames_to_tokens(frames: np.ndarray, T: int) -> np.ndarray:
+    """Token ids of the given frames, in order (frame f = tokens f*T .. f*T+T-1)."""
+    if len(frames) == 0:
+        return np.zeros(0, dtype=np.int64)
+    return (np.asarray(frames)[:, None] * T + np.arange(T)[None, :]).reshape(-1).astype(np.int64)
+
+
 def scoring_queries(q_cur: np.ndarray, stride: int) -> np.ndarray:
     """Rows 0, stride, 2*stride, ... of the chunk's queries (the scoring set)."""
     return q_cur[0::stride]
@@ -155,10 +162,19 @@ def advance(comp: np.ndarray, kept_count: int, seg_len: int, chunk: np.ndarray,
 
 def head_keep(*, granularity: str, dynamic: bool, mask_row, k: int, q_cur, k_hist,
               T: int, scale: float, score_stride: int = 1, q_score=None,
-              sink: int = 0, recent: int = 0, k_chunk=None):
+              sink: int = 0, recent: int = 0, k_chunk=None, token_static_mask: bool = False):
     """Selection for one (layer, head): (kept segment ids, segment scores or None).
-    k_chunk: include the chunk's own keys in the scoring normaliser."""
+    k_chunk: include the chunk's own keys in the scoring normaliser.
+    token_static_mask: static heads keep the tokens of a per-token mask (fixed
+    positions such as chunk-boundary tokens, Forcing-KV "关键模块" 1-2) and
+    every head's kept list is in tokens (a dynamic head's kept frames
+    expanded to their tokens)."""
     N = k_hist.shape[0]
+    if granularity == "frame" and token_static_mask:
+        if not dynamic:
+            return static_keep(mask_row), None
+        mass = segment_mass(scoring_queries(q_cur, score_stride), k_hist, T, scale, k_chunk)
+        return frames_to_tokens(top_k(mass, k), T), mass
     if granularity == "frame":
         if not dynamic:
             return static_keep(mask_row), None
@@ -212,4 +228,5 @@ def kept_rows(kept: np.ndarray, granularity: str, T: int) -> int:
 __all__: List[str] = [
     "static_keep", "scoring_queries", "segment_mass", "top_k", "participative_phi",
     "token_keep", "compact", "attention", "advance", "head_keep", "step", "kept_rows",
+    "frames_to_tokens",
 ]

@@ -93,7 +93,8 @@ def check_step(w, inputs_cpu, res, heads=None, rows=None, check_comp=True):
     x = HeadView(inputs_cpu)
     L, H = w.L, w.H
     todo = heads if heads is not None else [(l, h) for l in range(L) for h in range(H)]
-    seg_len = w.T if w.granularity == "frame" else 1
+    token_mask = getattr(w, "static_token_mask", False)
+    seg_len = w.T if (w.granularity == "frame" and not token_mask) else 1
     assert res["status"][0] == 0, f"device status {res['status']}"
     stats = {"attn_max": 0.0, "attn_mean": 0.0, "score_rel": 0.0, "sel_exact": 0, "sel_tie": 0}
     for (l, h) in todo:
@@ -108,7 +109,8 @@ def check_step(w, inputs_cpu, res, heads=None, rows=None, check_comp=True):
             T=w.T, scale=w.scale, score_stride=w.score_stride,
             q_score=None if "q_score" not in inputs_cpu else x("q_score", l, h),
             sink=w.sink_tokens, recent=w.recent_tokens,
-            k_chunk=x("k_cur", l, h) if getattr(w, "score_with_chunk", False) else None)
+            k_chunk=x("k_cur", l, h) if getattr(w, "score_with_chunk", False) else None,
+            token_static_mask=token_mask)
         kept_g = gpu_kept(res, l, h)
         if score_o is not None and len(score_o) > 0:
             sg = res["seg_score"][l, h].numpy().astype(np.float64)
@@ -122,6 +124,11 @@ def check_step(w, inputs_cpu, res, heads=None, rows=None, check_comp=True):
             assert np.array_equal(kept_g[:w.sink_tokens], np.arange(w.sink_tokens))
             assert np.array_equal(kept_g[len(kept_g) - w.recent_tokens:],
                                   np.arange(w.N - w.recent_tokens, w.N))
+        elif token_mask and dynamic:
+            # token lists of whole frames: compare the frames, then the expansion
+            fr_g = np.unique(kept_g // w.T)
+            assert np.array_equal(kept_g, orc.frames_to_tokens(fr_g, w.T)), f"{where}: not whole frames"
+            exact = check_selection(np.unique(kept_o // w.T), score_o, fr_g, k_sel, where)
         else:
             exact = check_selection(kept_o, score_o, kept_g, k_sel, where)
         stats["sel_exact" if exact else "sel_tie"] += 1

@@ -120,3 +120,28 @@ def test_480p_scoring_normalised_with_the_chunk(cuda_device):
     heads = [(0, h) for h in range(w.H) if x["head_role"][0, h]]
     st = parity.check_step(w, x, res, rows=rows, heads=heads)
     print("480p score_with_chunk", st)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_static_token_masks(cuda_device, dtype):
+    """FKV_FLAG_STATIC_TOKEN_MASK: static heads keep fixed token positions; all
+    kept lists are token ids; the step, and the cache advance, run on tokens."""
+    w = wl.scaled(wl.get("480p"), name=f"tokmask_{dtype}", H=4, T=200, F=7, Fc=2, n_static=2,
+                  k_dynamic=3, score_stride=3, dtype=dtype, seed=24, static_token_mask=True)
+    x = wl.generate(w)
+    assert x["static_mask"].shape == (1, 4, 7 * 200)
+    res = parity.run_step(w, x)
+    parity.check_step(w, x, res)
+    for h in range(w.H):
+        if not x["head_role"][0, h]:
+            got = parity.gpu_kept(res, 0, h)
+            assert got.tolist() == np.flatnonzero(x["static_mask"][0, h].numpy()).tolist()
+
+
+def test_480p_static_token_masks(cuda_device):
+    w = wl.scaled(wl.get("480p"), static_token_mask=True)
+    x = wl.generate(w)
+    res = parity.run_step(w, x)
+    rows = wl.sample_rows(w.Lq, 16, seed=9)
+    st = parity.check_step(w, x, res, rows=rows)
+    print("480p static token masks", st, res["kept_cnt"].tolist())

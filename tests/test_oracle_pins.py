@@ -331,3 +331,19 @@ def test_mass_with_chunk_in_the_normaliser_closed_form():
         exp.append(tot)
     np.testing.assert_allclose(got, exp, rtol=1e-13)
     assert got.sum() < len(a)  # part of each row's mass now sits on the chunk
+
+
+def test_token_static_mask_keeps_tokens_and_expands_frames():
+    T = 3
+    mask = np.zeros(12, np.uint8)
+    mask[[0, 2, 5, 11]] = 1
+    kept, sc = orc.head_keep(granularity="frame", dynamic=False, mask_row=mask, k=0,
+                             q_cur=np.zeros((2, 4)), k_hist=np.zeros((12, 4)), T=T, scale=1.0,
+                             token_static_mask=True)
+    assert kept.tolist() == [0, 2, 5, 11] and sc is None
+    assert orc.frames_to_tokens(np.array([1, 3]), T).tolist() == [3, 4, 5, 9, 10, 11]
+    rng = np.random.default_rng(16)
+    q, k = rng.standard_normal((3, 4)), rng.standard_normal((12, 4))
+    kept, mass = orc.head_keep(granularity="frame", dynamic=True, mask_row=mask, k=2, q_cur=q,
+                               k_hist=k, T=T, scale=0.5, token_static_mask=True)
+    assert kept.tolist() == orc.frames_to_tokens(orc.top_k(mass, 2), T).tolist()

@@ -65,7 +65,7 @@ def algorithmic(w, kept_cnt, head_role):
     scoring (frame): 2 * n_s * N * D per dynamic head (QK^T), K read once;
     scoring (token): K candidates read once (GEMV) + q_score read once;
     compaction: kept rows of K and V read once and written once."""
-    seg_len = w.T if w.granularity == "frame" else 1
+    seg_len = w.T if (w.granularity == "frame" and not w.static_token_mask) else 1
     rows = kept_cnt.to(torch.int64) * seg_len
     keys = rows + w.Lq
     elem = 2 if w.dtype == "bf16" else 4
@@ -321,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
     # policies: compress at every denoising step, or once per chunk and reuse
     # the selection (attention alone for the later steps).
     lifecycle = None
-    if w.granularity == "frame" and w.L == 1:
+    if w.granularity == "frame" and not w.static_token_mask and w.L == 1:
         n_den = 4
         kept = int(outs["kept_cnt"].min())
         window = min(kept, w.F - w.Fc) + w.Fc
@@ -448,8 +448,10 @@ def cpu_baseline(w, x_cpu, budget_s=15.0):
             mask_row=x["static_mask"][l, h].numpy(), k=int(x["k_per_head"][l, h]),
             q_cur=f64("q_cur"), k_hist=f64("k_hist"), T=w.T, scale=w.scale,
             score_stride=w.score_stride, q_score=f64("q_score") if "q_score" in x else None,
-            sink=w.sink_tokens, recent=w.recent_tokens)
-        seg_len = w.T if w.granularity == "frame" else 1
+            sink=w.sink_tokens, recent=w.recent_tokens,
+            k_chunk=f64("k_cur") if w.score_with_chunk else None,
+            token_static_mask=w.static_token_mask)
+        seg_len = w.T if (w.granularity == "frame" and not w.static_token_mask) else 1
         keys = np.concatenate([orc.compact(f64("k_hist"), ks, seg_len), f64("k_cur")])
         vals = np.concatenate([orc.compact(f64("v_hist"), ks, seg_len), f64("v_cur")])
         orc.attention(f64("q_cur"), keys, vals, w.scale)

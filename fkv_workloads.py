@@ -136,6 +136,13 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
+# Options of the 480P workload (same inputs, other readings of the method).
+WORKLOADS["480p_chunknorm"] = dataclasses.replace(WORKLOADS["480p"], name="480p_chunknorm",
+                                                  score_with_chunk=True)
+WORKLOADS["480p_tokenmask"] = dataclasses.replace(WORKLOADS["480p"], name="480p_tokenmask",
+                                                  static_token_mask=True)
+
+
 def get(name: str) -> Workload:
     return WORKLOADS[name]
 

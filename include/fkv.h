@@ -251,6 +251,24 @@ int32_t fkv_attend_compressed(const fkv_params_t* p, const void* q_cur, const vo
                               const void* v_cur, const void* k_comp, const void* v_comp,
                               const int32_t* kept_cnt, void* out, void* ws, void* stream);
 
+/* Step 4 with temporal RoPE re-positioning of the kept keys (frame mode,
+ * frame masks): the copy of fkv_compact_gather, except that the p-th of the
+ * cnt kept frames of a head moves from frame kept_idx[p] to frame
+ * F - cnt + p (the kept frames close up, ending right before the chunk), and
+ * the temporal band of its keys -- the first n_pairs pairs of adjacent dims
+ * (k[2i], k[2i+1]) taken as complex numbers -- is rotated by the angle
+ * omega[i] * ((F - cnt + p) - kept_idx[p]); other dims and the values are
+ * copied unchanged.  Deep Forcing (bxzpzcl.cn/news/2125000, section 2.2.2)
+ * rotates cached keys' time component by the phase exp(i omega_t delta) when
+ * their temporal offset changes (section 3.2 item 3: also for selected
+ * tokens).  omega: device float[n_pairs], the model's temporal RoPE
+ * frequencies; 0 <= 2*n_pairs <= D.  Rotation in fp32, rounded once to the
+ * activation dtype.  Token mode / token masks: FKV_ERR_UNSUPPORTED. */
+int32_t fkv_compact_gather_rope(const fkv_params_t* p, const void* k_hist, const void* v_hist,
+                                const int32_t* kept_idx, const int32_t* kept_cnt,
+                                const float* omega, int32_t n_pairs, void* k_comp, void* v_comp,
+                                void* ws, void* stream);
+
 /* Cache lifecycle: the history cache for the next chunk.  For each (l, h),
  * k_next[l][h] = the last (out_segments - chunk_segs) kept segments of the
  * compressed cache (rows of k_comp, in order), followed by the Lq rows of the

@@ -30,6 +30,7 @@ __all__ = [
     "FkvError", "Params", "make_params", "params_for", "sizes", "allocate", "score_segments",
     "select_topk", "compact_gather", "attend_compressed", "step", "read_status", "library",
     "step_launches", "make_step_io", "score_segments_noalloc", "cache_advance",
+    "compact_gather_rope",
 ]
 
 
@@ -245,6 +246,23 @@ def attend_compressed(p: Params, q_cur, k_cur, v_cur, k_comp, v_comp, kept_cnt, 
         _ptr(v_comp, "v_comp", dt, n["comp"]), _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]),
         _ptr(out, "out", dt, n["act_cur"]), _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
     _check(st, "fkv_attend_compressed")
+
+
+def compact_gather_rope(p: Params, k_hist, v_hist, kept_idx, kept_cnt, omega, k_comp, v_comp, ws,
+                        stream=None):
+    """Compaction with temporal RoPE re-positioning of the kept keys
+    (fkv_compact_gather_rope); omega: float32 CUDA tensor of the temporal
+    RoPE frequencies, one per rotated dim pair."""
+    n, dt = _shapes(p), _act_dtype(p)
+    n_pairs = 0 if omega is None else int(omega.numel())
+    st = _lib.load().fkv_compact_gather_rope(
+        ctypes.byref(p), _ptr(k_hist, "k_hist", dt, n["act_hist"]),
+        _ptr(v_hist, "v_hist", dt, n["act_hist"]), _ptr(kept_idx, "kept_idx", torch.int32, n["kept"]),
+        _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]),
+        _ptr(omega, "omega", torch.float32, n_pairs, optional=n_pairs == 0), n_pairs,
+        _ptr(k_comp, "k_comp", dt, n["comp"]), _ptr(v_comp, "v_comp", dt, n["comp"]),
+        _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
+    _check(st, "fkv_compact_gather_rope")
 
 
 def cache_advance(p: Params, k_comp, v_comp, kept_cnt, k_cur, v_cur, out_segments: int, k_next,

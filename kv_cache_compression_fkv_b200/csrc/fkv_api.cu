@@ -342,6 +342,26 @@ int32_t fkv_attend_compressed(const fkv_params_t* p, const void* q_cur, const vo
                    static_cast<cudaStream_t>(stream));
 }
 
+int32_t fkv_compact_gather_rope(const fkv_params_t* p, const void* k_hist, const void* v_hist,
+                                const int32_t* kept_idx, const int32_t* kept_cnt,
+                                const float* omega, int32_t n_pairs, void* k_comp, void* v_comp,
+                                void* ws, void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (d.token || d.static_token_mask) return FKV_ERR_UNSUPPORTED;  // frames only
+  if (n_pairs < 0 || 2 * n_pairs > d.D) return FKV_ERR_SHAPE;
+  if (((!k_hist || !v_hist) && d.N > 0) || (!kept_idx && d.max_kept > 0) || !kept_cnt ||
+      ((!k_comp || !v_comp) && d.comp_rows > 0) || (n_pairs > 0 && !omega))
+    return FKV_ERR_INVALID_ARG;
+  if (!aligned16(k_hist) || !aligned16(v_hist) || !aligned16(k_comp) || !aligned16(v_comp))
+    return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  return cuda_status(launch_gather_rope(d, k_hist, v_hist, kept_idx, kept_cnt, omega, n_pairs,
+                                        k_comp, v_comp, status_ptr(ws),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 int32_t fkv_cache_advance(const fkv_params_t* p, const void* k_comp, const void* v_comp,
                           const int32_t* kept_cnt, const void* k_cur, const void* v_cur,
                           int64_t out_segments, void* k_next, void* v_next, void* ws,

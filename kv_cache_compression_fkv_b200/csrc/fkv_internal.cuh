@@ -100,6 +100,10 @@ cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_
                                 const void* v_cur, const void* k_comp, const void* v_comp,
                                 const int32_t* kept_cnt, void* out, int32_t* status,
                                 cudaStream_t s);
+cudaError_t launch_gather_rope(const Dims& d, const void* k_hist, const void* v_hist,
+                               const int32_t* kept_idx, const int32_t* kept_cnt,
+                               const float* omega, int32_t n_pairs, void* k_comp, void* v_comp,
+                               int32_t* status, cudaStream_t s);
 cudaError_t launch_advance(const Dims& d, int64_t out_segments, const void* k_comp,
                            const void* v_comp, const int32_t* kept_cnt, const void* k_cur,
                            const void* v_cur, void* k_next, void* v_next, int32_t* status,

@@ -125,6 +125,40 @@ def compact(kv_hist: np.ndarray, kept: np.ndarray, seg_len: int) -> np.ndarray:
     return np.concatenate([kv_hist[s * seg_len:(s + 1) * seg_len] for s in kept], axis=0)
 
 
+def rope_shift(keys: np.ndarray, omega: np.ndarray, delta: float) -> np.ndarray:
+    """Temporal RoPE re-positioning of keys by delta frames.
+
+    Deep Forcing (bxzpzcl.cn/news/2125000), section 2.2.2 (and 3.2 item 3 for
+    selected tokens): the time component of a cached key is multiplied by the
+    phase exp(i * omega_t * delta).  Read as: the first len(omega) pairs of
+    adjacent dims (k[2i], k[2i+1]) are complex numbers k[2i] + i k[2i+1], each
+    rotated by the angle omega[i] * delta; the other dims are unchanged.
+    keys [rows][D] -> [rows][D].
+    """
+    out = np.array(keys, dtype=np.float64, copy=True)
+    n = len(omega)
+    ang = np.asarray(omega, dtype=np.float64) * float(delta)
+    c, s = np.cos(ang), np.sin(ang)
+    x0, x1 = out[:, 0:2 * n:2].copy(), out[:, 1:2 * n:2].copy()
+    out[:, 0:2 * n:2] = x0 * c - x1 * s
+    out[:, 1:2 * n:2] = x0 * s + x1 * c
+    return out
+
+
+def compact_repositioned(k_hist: np.ndarray, kept: np.ndarray, T: int, F: int,
+                         omega: np.ndarray) -> np.ndarray:
+    """Compressed keys with their temporal position re-assigned: the p-th of
+    cnt kept frames moves from frame kept[p] to frame F - cnt + p (the kept
+    frames close up, ending right before the chunk at frame F), and its keys
+    are rotated by rope_shift with delta = (F - cnt + p) - kept[p]."""
+    cnt = len(kept)
+    parts = [rope_shift(k_hist[f * T:(f + 1) * T], omega, (F - cnt + p) - f)
+             for p, f in enumerate(kept)]
+    if not parts:
+        return k_hist[:0].copy()
+    return np.concatenate(parts, axis=0)
+
+
 def attention(q: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float) -> np.ndarray:
     """o_i = sum_j softmax_j(scale * q_i . k_j) v_j, max-subtracted, float64.
 
@@ -228,5 +262,5 @@ def kept_rows(kept: np.ndarray, granularity: str, T: int) -> int:
 __all__: List[str] = [
     "static_keep", "scoring_queries", "segment_mass", "top_k", "participative_phi",
     "token_keep", "compact", "attention", "advance", "head_keep", "step", "kept_rows",
-    "frames_to_tokens",
+    "frames_to_tokens", "rope_shift", "compact_repositioned",
 ]

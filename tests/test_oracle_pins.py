@@ -347,3 +347,35 @@ def test_token_static_mask_keeps_tokens_and_expands_frames():
     kept, mass = orc.head_keep(granularity="frame", dynamic=True, mask_row=mask, k=2, q_cur=q,
                                k_hist=k, T=T, scale=0.5, token_static_mask=True)
     assert kept.tolist() == orc.frames_to_tokens(orc.top_k(mass, 2), T).tolist()
+
+
+def test_rope_shift_rotation_identities():
+    rng = np.random.default_rng(17)
+    k = rng.standard_normal((5, 8))
+    om = np.array([0.5, 1.25, 3.0])
+    # rotating by a then by b is rotating by a + b; by -d undoes d
+    np.testing.assert_allclose(orc.rope_shift(orc.rope_shift(k, om, 2.0), om, 3.0),
+                               orc.rope_shift(k, om, 5.0), atol=1e-12)
+    np.testing.assert_allclose(orc.rope_shift(orc.rope_shift(k, om, 4.0), om, -4.0), k, atol=1e-12)
+    # a quarter turn maps (x0, x1) to (-x1, x0); dims past the band are untouched
+    q = orc.rope_shift(k, np.array([math.pi / 2]), 1.0)
+    np.testing.assert_allclose(q[:, 0], -k[:, 1], atol=1e-15)
+    np.testing.assert_allclose(q[:, 1], k[:, 0], atol=1e-15)
+    assert np.array_equal(q[:, 2:], k[:, 2:])
+    # pair norms are preserved
+    r = orc.rope_shift(k, om, 7.0)
+    for i in range(3):
+        np.testing.assert_allclose(np.hypot(r[:, 2 * i], r[:, 2 * i + 1]),
+                                   np.hypot(k[:, 2 * i], k[:, 2 * i + 1]), rtol=1e-13)
+    # delta 0 (a frame that keeps its place) is the identity
+    np.testing.assert_allclose(orc.rope_shift(k, om, 0.0), k, atol=0)
+
+
+def test_compact_repositioned_closes_the_gaps():
+    T, F, D = 2, 6, 4
+    k = np.arange(F * T * D, dtype=np.float64).reshape(F * T, D)
+    om = np.array([0.3])
+    got = orc.compact_repositioned(k, np.array([1, 4, 5]), T, F, om)
+    # frames 1, 4, 5 move to 3, 4, 5: deltas 2, 0, 0
+    np.testing.assert_allclose(got[:2], orc.rope_shift(k[2:4], om, 2.0), atol=1e-12)
+    assert np.array_equal(got[2:], k[8:12])

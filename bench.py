@@ -238,7 +238,10 @@ def run_ours(args, rank, world, local_rank):
     clocks = clk.summary()
 
     # ---- per-kernel breakdown: the same kernels through the four entry points
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    rope = w.granularity == "frame" and not w.static_token_mask
+    # temporal RoPE band of the re-positioning compaction: 22 pairs (44 dims)
+    omega = (10000.0 ** (-torch.arange(22, dtype=torch.float32) / 22)).to(dev)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
     barrier()
     for i in range(args.steps):
         flush.fill_(i & 0xFF)
@@ -256,10 +259,14 @@ def run_ours(args, rank, world, local_rank):
         fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"], outs["v_comp"],
                               outs["kept_cnt"], outs["out"], outs["ws"])
         e[4].record(stream)
+        if rope:
+            fkv.compact_gather_rope(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
+                                    omega, outs["k_comp"], outs["v_comp"], outs["ws"])
+        e[5].record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
-            for j, n in enumerate(["score", "select", "gather", "attend"])}
+            for j, n in enumerate(["score", "select", "gather", "attend", "gather_rope"])}
 
     # ---- e2e: host buffers in, result out, through the same call.  Every step
     # copies its inputs from pinned host memory (H2D stream), runs fkv_step
@@ -381,6 +388,10 @@ def run_ours(args, rank, world, local_rank):
                            "frac_tensor": round(score_tfs / peaks["bf16_tflops"], 4),
                            "frac_hbm": round(score_gbs / peaks["hbm_gbs"], 4)},
         "select_topk": {"ms": round(part["select"], 4)},
+        "compact_gather_rope": ({"ms": round(part["gather_rope"], 4),
+                                 "GB/s": round(alg["gather_bytes"] / (part["gather_rope"] * 1e-3) / 1e9, 1),
+                                 "frac_hbm": round(alg["gather_bytes"] / (part["gather_rope"] * 1e-3) / 1e9
+                                                   / peaks["hbm_gbs"], 4)} if rope else None),
         "compact_gather": {"ms": round(part["gather"], 4), "GB/s": round(gather_gbs, 1),
                            "frac_hbm": round(gather_gbs / peaks["hbm_gbs"], 4),
                            "frac_hbm_spec": round(gather_gbs / SPEC_HBM_GBS, 4)},

@@ -11,6 +11,9 @@ Modules
               (attention may be evaluated on a subset of query rows).
   fkv_loops   pure-Python loops over ``math``; tiny inputs only.  A second,
               independent spelling of the same definitions.
+  fkv_fp8     the e4m3 compressed cache: codes and per-segment scales (fp32
+              decisions, as the kernels take them), dequantisation, and the
+              error model of an fp8 tensor-core attention.
 
 Sources (page title and section):
   Forcing-KV (ai-feeds.com/i/paper/2605.09681): "关键模块" items 2 (static

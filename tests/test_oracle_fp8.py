@@ -1,0 +1,158 @@
+"""Pins of the fp8 (e4m3) compressed-cache oracle against the format's
+definition, a library conversion, closed forms and a simulation.
+
+Forcing-KV (ai-feeds.com/i/paper/2605.09681), "与现有产品/工作流的接口"
+item 3: the compression composes with KV quantization; the format and scale
+granularity are the reading stated in ``oracle.fkv_fp8``.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import fkv_fp8 as f8
+from oracle import fkv_oracle as fo
+
+
+def test_decode_table_landmarks():
+    # exponent field 0: multiples of 2^-9; field 7 mantissa 0: 1.0; 0x7e: 448
+    cases = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6,
+             0x38: 1.0, 0x39: 1.125, 0x3F: 1.875, 0x40: 2.0, 0x7E: 448.0, 0x77: 240.0,
+             0xB8: -1.0, 0xFE: -448.0}
+    for c, v in cases.items():
+        assert f8.e4m3_decode(np.uint8(c)) == v, hex(c)
+    assert np.isnan(f8.e4m3_decode(np.uint8(0x7F))) and np.isnan(f8.e4m3_decode(np.uint8(0xFF)))
+
+
+def test_encode_inverts_decode_on_every_finite_code():
+    codes = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+    vals = f8.e4m3_decode(codes).astype(np.float32)
+    back = f8.e4m3_encode(vals)
+    assert np.array_equal(back, codes)
+    # 254 finite codes, strictly increasing magnitude within a sign
+    pos = f8.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    assert np.all(np.diff(pos) > 0) and pos[-1] == 448.0
+
+
+def test_ties_to_even_and_saturation():
+    x = np.array([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 5 * 2.0 ** -10, 464.0, 465.0,
+                  1e6, -500.0, np.inf, 17 * 2.0 ** -11], dtype=np.float32)
+    want = [0x38, 0x3A, 0x00, 0x02, 0x02, 0x7E, 0x7E, 0x7E, 0xFE, 0x7E, 0x04]
+    assert f8.e4m3_encode(x).tolist() == want
+
+
+def test_encode_matches_torch_float8_e4m3fn_in_range():
+    # torch's cast is round-to-nearest-even; it returns NaN instead of
+    # saturating, so the comparison stays within +-448.
+    rng = np.random.default_rng(11)
+    mag = np.exp2(rng.uniform(-12, np.log2(448.0), 200_000)).astype(np.float32)
+    x = (mag * rng.choice([-1.0, 1.0], mag.size)).astype(np.float32)
+    x = np.concatenate([x, np.float32([0.0, -0.0, 448.0, -448.0])])
+    ours = f8.e4m3_encode(x)
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, lib)
+
+
+def test_rounding_error_bounds():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(100_000) * 30).astype(np.float32)
+    x = x[np.abs(x) <= 448]
+    err = np.abs(f8.e4m3_decode(f8.e4m3_encode(x)) - x.astype(np.float64))
+    normal = np.abs(x) >= 2.0 ** -6
+    assert np.all(err[normal] <= 2.0 ** -4 * np.abs(x[normal]) * (1 + 1e-12))
+    assert np.all(err[~normal] <= 2.0 ** -10)
+
+
+def test_quantize_block_scale_and_extremes():
+    rng = np.random.default_rng(5)
+    x = (rng.standard_normal((40, 128)) * 2.5).astype(np.float32)
+    codes, s = f8.quantize_block(x)
+    amax = np.float32(np.abs(x).max())
+    i = np.unravel_index(np.argmax(np.abs(x)), x.shape)
+    assert codes[i] in (0x7E, 0xFE)                  # the largest element lands on +-448
+    assert s == np.float32(amax / np.float32(448.0))
+    assert abs(float(s) * 448.0 - float(amax)) <= float(np.spacing(amax))
+    deq = f8.e4m3_decode(codes) * float(s)
+    assert np.all(np.abs(deq) <= float(amax) * (1 + 2.0 ** -22))
+    # relative error of normal-range elements (x * inv >= 2^-6)
+    big = np.abs(x) >= float(amax) / 448.0 * 2.0 ** -6 * 1.01
+    assert np.all(np.abs(deq - x)[big] <= (2.0 ** -4 + 2.0 ** -20) * np.abs(x)[big])
+    z, sz = f8.quantize_block(np.zeros((3, 8), np.float32))
+    assert sz == 1.0 and not z.any()
+
+
+def test_exactly_representable_cache_is_lossless():
+    # Every segment holds e4m3 values with 448 as its largest magnitude, so
+    # the scale is exactly 1, the codes are the values, and fp8 attention over
+    # the dequantised cache is the exact attention over the original values.
+    rng = np.random.default_rng(9)
+    T, D, F = 24, 64, 5
+    codes = rng.integers(0, 0x7E, size=(F * T, D), dtype=np.int64).astype(np.uint8)
+    codes |= (rng.integers(0, 2, size=codes.shape) << 7).astype(np.uint8)
+    codes[::T, 0] = 0x7E
+    k = f8.e4m3_decode(codes).astype(np.float32)
+    kc, sk = f8.quantize_segments(k, T)
+    assert np.array_equal(kc, codes) and np.all(sk == 1.0)
+    q = rng.standard_normal((7, D)) * 0.01
+    out8 = fo.attention(q, f8.dequantize(kc, sk, T), f8.dequantize(kc, sk, T), 0.125)
+    out = fo.attention(q, k.astype(np.float64), k.astype(np.float64), 0.125)
+    assert np.array_equal(out8, out)
+
+
+def test_compact_quantized_is_gather_then_quantize():
+    rng = np.random.default_rng(2)
+    T, D, F = 16, 32, 6
+    k = rng.standard_normal((F * T, D)).astype(np.float32) * rng.uniform(0.1, 4, (F * T, 1)).astype(np.float32)
+    v = rng.standard_normal((F * T, D)).astype(np.float32)
+    kept = np.array([0, 2, 3, 5])
+    kc, sk, vc, sv = f8.compact_quantized(k, v, kept, T)
+    kc2, sk2 = f8.quantize_segments(fo.compact(k, kept, T), T)
+    vc2, sv2 = f8.quantize_segments(fo.compact(v, kept, T), T)
+    assert np.array_equal(kc, kc2) and np.array_equal(sk, sk2)
+    assert np.array_equal(vc, vc2) and np.array_equal(sv, sv2)
+    # per-segment: one segment's scale does not depend on the others
+    _, s_alone = f8.quantize_block(k[2 * T:3 * T])
+    assert sk[1] == s_alone
+
+
+def test_quantize_rows_per_row_scale():
+    rng = np.random.default_rng(4)
+    x = (rng.standard_normal((9, 128)) * np.arange(1, 10)[:, None]).astype(np.float32)
+    codes, s = f8.quantize_rows(x)
+    for r in range(9):
+        c1, s1 = f8.quantize_block(x[r])
+        assert np.array_equal(codes[r], c1) and s[r] == s1
+
+
+def _simulated_fp8_attention(q, keys, v_codes, sv_key, scale, lag_log2):
+    """The evaluation model of attention_tolerance, spelled out directly:
+    probabilities relative to (true max - lag) in base 2, times sv/max(sv),
+    rounded to e4m3; fp64 accumulation; bf16 output rounding."""
+    sv_max = sv_key.max()
+    logits = (q @ keys.T) * scale * np.log2(np.e)
+    m = logits.max(axis=1, keepdims=True) - lag_log2
+    p = np.exp2(logits - m)
+    p_scaled = (p * (sv_key / sv_max)[None, :]).astype(np.float32)
+    p8 = f8.e4m3_decode(f8.e4m3_encode(p_scaled))
+    acc = p8 @ f8.e4m3_decode(v_codes)
+    out = acc * sv_max / p.sum(axis=1, keepdims=True)
+    return torch.from_numpy(out).to(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("lag", [0.0, 3.5, 7.9])
+def test_tolerance_covers_simulated_evaluation(lag):
+    rng = np.random.default_rng(int(lag * 10) + 1)
+    T, D, F = 64, 64, 8
+    q = rng.standard_normal((32, D))
+    k = rng.standard_normal((F * T, D)) * 1.5
+    v = (rng.standard_normal((F * T, D)) * rng.uniform(0.5, 3, (F * T, 1))).astype(np.float32)
+    vc, sv = f8.quantize_segments(v, T)
+    sv_key = np.repeat(sv.astype(np.float64), T)
+    vals = f8.dequantize(vc, sv, T)
+    ref = fo.attention(q, k, vals, 0.125)
+    tol = f8.attention_tolerance(q, k, vc, sv_key, 0.125, ref)
+    sim = _simulated_fp8_attention(q, k, vc, sv_key, 0.125, lag)
+    err = np.abs(sim - ref)
+    assert np.all(err <= tol)
+    # and the bound is not vacuous: a dropped V scale breaks it
+    wrong = _simulated_fp8_attention(q, k, vc, np.ones_like(sv_key), 0.125, lag) * sv_key.max()
+    assert np.any(np.abs(wrong - ref) > tol)

@@ -279,3 +279,27 @@ __all__: Sequence[str] = (
     "Workload", "WORKLOADS", "STATIC_FRAMES_18", "get", "scaled", "generate",
     "as_float64", "sample_rows",
 )
+
+
+def random_kept(w: Workload, seed: int, n_keep: Optional[int] = None):
+    """Seeded kept-frame lists for exercising the compaction and attention on
+    their own: per (layer, head) an ascending random subset of the F history
+    frames, padded with -1.  Its size is n_keep (default: a random count);
+    head (0, 0) keeps nothing and, when there are two or more heads, head
+    (0, 1) keeps every frame.  Returns (kept_idx int32 [L][H][F], kept_cnt
+    int32 [L][H])."""
+    rng = np.random.default_rng(seed)
+    idx = np.full((w.L, w.H, w.F), -1, dtype=np.int32)
+    cnt = np.zeros((w.L, w.H), dtype=np.int32)
+    for l in range(w.L):
+        for h in range(w.H):
+            if (l, h) == (0, 0):
+                c = 0
+            elif (l, h) == (0, 1):
+                c = w.F
+            else:
+                c = int(rng.integers(0, w.F + 1)) if n_keep is None else n_keep
+            frames = np.sort(rng.choice(w.F, size=c, replace=False)) if c else np.zeros(0, int)
+            idx[l, h, :c] = frames
+            cnt[l, h] = c
+    return torch.from_numpy(idx), torch.from_numpy(cnt)

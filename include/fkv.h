@@ -53,7 +53,8 @@
 extern "C" {
 #endif
 
-#define FKV_ABI_VERSION 2
+/* 3: adds fkv_fp8_cache_t and the three *_fp8 entry points. */
+#define FKV_ABI_VERSION 3
 
 typedef enum fkv_status {
   FKV_OK = 0,
@@ -294,6 +295,72 @@ int32_t fkv_cache_advance(const fkv_params_t* p, const void* k_comp, const void*
 /* Steps 1-5 in one call: score (dynamic / token heads), select, compact,
  * attend, all enqueued on `stream` in that order. */
 int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void* stream);
+
+/* ---- FP8 (e4m3) compressed cache ------------------------------------------
+ * Forcing-KV (ai-feeds.com/i/paper/2605.09681), "与现有产品/工作流的接口" item
+ * 3: the compression composes with KV quantization; the pages fix no format.
+ * Reading: OCP FP8 E4M3 (largest finite 448), round to nearest even,
+ * saturating; one fp32 scale per (l, h, segment) for K and one for V, where a
+ * segment is a kept history frame or a frame of the current chunk, and one per
+ * query row for Q.  Scale s = amax / 448 over the block (1 for an all-zero
+ * block); code = e4m3(x * (448 / amax)), each division and the product one
+ * correctly rounded fp32 operation.  The value a code stands for is
+ * e4m3(code) * s.
+ *
+ * Operands of the fp8 attention, all device memory owned by the caller, all
+ * code arrays row-major with D = 128 bytes per row and 16-byte aligned:
+ *   k_comp, v_comp  uint8 [L*H][comp_rows][D]  kept history rows, segment p
+ *                   (the p-th kept frame) in rows [p*T, (p+1)*T)
+ *   k_comp_scale, v_comp_scale  float [L*H][F]  scale of kept segment p
+ *   k_cur, v_cur    uint8 [L*H][Lq][D]         the chunk's own rows
+ *   k_cur_scale, v_cur_scale    float [L*H][Fc] scale of chunk frame g
+ *   q_cur           uint8 [L*H][Lq][D]         the chunk's queries
+ *   q_scale         float [L*H][Lq]            scale of query row r
+ * Supported: bf16 activations, head_dim 128, frame granularity with frame
+ * masks; otherwise FKV_ERR_UNSUPPORTED.  The attention also needs
+ * frame_tokens >= 128 (a 128-key block spans at most two segments). */
+typedef struct fkv_fp8_cache {
+  void* k_comp;
+  void* v_comp;
+  float* k_comp_scale;
+  float* v_comp_scale;
+  void* k_cur;
+  void* v_cur;
+  float* k_cur_scale;
+  float* v_cur_scale;
+  void* q_cur;
+  float* q_scale;
+} fkv_fp8_cache_t;
+
+/* Step 4 into the fp8 cache: for each (l, h) and p < kept_cnt[l][h], the
+ * frame kept_idx[l][h][p] of k_hist / v_hist (bf16 [L*H][F*T][D]) is
+ * quantized as one segment into rows [p*T, (p+1)*T) of c->k_comp / c->v_comp
+ * and its scales into c->k_comp_scale[l][h][p] / c->v_comp_scale[l][h][p].
+ * Rows and scales of segments p >= kept_cnt are not written.  A kept_cnt or
+ * kept_idx entry out of range is reported as FKV_ERR_DEVICE_ARG through the
+ * workspace status and that segment skipped.  c: host struct, only the
+ * k_comp / v_comp / *_comp_scale members are used. */
+int32_t fkv_compact_gather_fp8(const fkv_params_t* p, const void* k_hist, const void* v_hist,
+                               const int32_t* kept_idx, const int32_t* kept_cnt,
+                               const fkv_fp8_cache_t* c, void* ws, void* stream);
+
+/* The chunk's own operands in fp8: k_cur / v_cur (bf16 [L*H][Lq][D]) frame by
+ * frame into c->k_cur / c->v_cur with per-frame scales, q_cur (bf16
+ * [L*H][Lq][D]) row by row into c->q_cur / c->q_scale.  c: host struct, only
+ * the *_cur members and q_scale are used. */
+int32_t fkv_quantize_chunk_fp8(const fkv_params_t* p, const void* q_cur, const void* k_cur,
+                               const void* v_cur, const fkv_fp8_cache_t* c, void* ws,
+                               void* stream);
+
+/* Step 5 over the fp8 cache: out (bf16 [L*H][Lq][D]) = softmax attention of
+ * the dequantised queries over the dequantised keys = kept rows
+ * [0, kept_cnt*T) of k_comp then the Lq rows of k_cur, with values likewise,
+ * scale p->scale.  Tensor cores (kind::f8f6f4) with fp32 accumulation; the
+ * probabilities are rounded to e4m3 before the P.V product (after a per-head
+ * rescale by v_scale / max v_scale), so the result differs from the exact
+ * attention over the dequantised cache by that rounding. */
+int32_t fkv_attend_compressed_fp8(const fkv_params_t* p, const fkv_fp8_cache_t* c,
+                                  const int32_t* kept_cnt, void* out, void* ws, void* stream);
 
 #ifdef __cplusplus
 }

@@ -321,6 +321,82 @@ def step(p: Params, inputs: Dict[str, torch.Tensor], outputs: Dict[str, torch.Te
     _check(st, "fkv_step")
 
 
+def allocate_fp8(p: Params, device="cuda") -> Dict[str, torch.Tensor]:
+    """Buffers of the e4m3 compressed cache (fkv_fp8_cache_t): codes as uint8,
+    scales as float32 (k_comp_scale / v_comp_scale: one per kept segment,
+    k_cur_scale / v_cur_scale: one per chunk frame, q_scale: one per query)."""
+    L, H, D = p.num_layers, p.num_heads, p.head_dim
+    Lq = p.chunk_frames * p.frame_tokens
+    u8, f32 = torch.uint8, torch.float32
+    return {
+        "k_comp": torch.empty((L, H, p.comp_rows, D), dtype=u8, device=device),
+        "v_comp": torch.empty((L, H, p.comp_rows, D), dtype=u8, device=device),
+        "k_comp_scale": torch.empty((L, H, p.hist_frames), dtype=f32, device=device),
+        "v_comp_scale": torch.empty((L, H, p.hist_frames), dtype=f32, device=device),
+        "k_cur": torch.empty((L, H, Lq, D), dtype=u8, device=device),
+        "v_cur": torch.empty((L, H, Lq, D), dtype=u8, device=device),
+        "k_cur_scale": torch.empty((L, H, p.chunk_frames), dtype=f32, device=device),
+        "v_cur_scale": torch.empty((L, H, p.chunk_frames), dtype=f32, device=device),
+        "q_cur": torch.empty((L, H, Lq, D), dtype=u8, device=device),
+        "q_scale": torch.empty((L, H, Lq), dtype=f32, device=device),
+    }
+
+
+def make_fp8_cache(p: Params, c: Dict[str, torch.Tensor]) -> _lib.Fp8Cache:
+    """fkv_fp8_cache_t over the tensors of allocate_fp8 (shapes checked)."""
+    L, H, D = p.num_layers, p.num_heads, p.head_dim
+    Lq = p.chunk_frames * p.frame_tokens
+    need = {
+        "k_comp": (torch.uint8, L * H * p.comp_rows * D), "v_comp": (torch.uint8, L * H * p.comp_rows * D),
+        "k_comp_scale": (torch.float32, L * H * p.hist_frames),
+        "v_comp_scale": (torch.float32, L * H * p.hist_frames),
+        "k_cur": (torch.uint8, L * H * Lq * D), "v_cur": (torch.uint8, L * H * Lq * D),
+        "k_cur_scale": (torch.float32, L * H * p.chunk_frames),
+        "v_cur_scale": (torch.float32, L * H * p.chunk_frames),
+        "q_cur": (torch.uint8, L * H * Lq * D), "q_scale": (torch.float32, L * H * Lq),
+    }
+    fp = _lib.Fp8Cache()
+    for name in _lib.FP8_CACHE_FIELDS:
+        dt, n = need[name]
+        setattr(fp, name, _ptr(c.get(name), name, dt, n, optional=n == 0))
+    return fp
+
+
+def compact_gather_fp8(p: Params, k_hist, v_hist, kept_idx, kept_cnt, cache, ws, stream=None):
+    """Step 4 into the e4m3 cache (fkv_compact_gather_fp8): kept frames
+    quantised per segment into cache["k_comp"] / ["v_comp"] and their scales."""
+    n, dt = _shapes(p), _act_dtype(p)
+    fp = make_fp8_cache(p, cache)
+    st = _lib.load().fkv_compact_gather_fp8(
+        ctypes.byref(p), _ptr(k_hist, "k_hist", dt, n["act_hist"]),
+        _ptr(v_hist, "v_hist", dt, n["act_hist"]), _ptr(kept_idx, "kept_idx", torch.int32, n["kept"]),
+        _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]), ctypes.byref(fp),
+        _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
+    _check(st, "fkv_compact_gather_fp8")
+
+
+def quantize_chunk_fp8(p: Params, q_cur, k_cur, v_cur, cache, ws, stream=None):
+    """The chunk's own operands in e4m3 (fkv_quantize_chunk_fp8): K / V per
+    frame, Q per row."""
+    n, dt = _shapes(p), _act_dtype(p)
+    fp = make_fp8_cache(p, cache)
+    st = _lib.load().fkv_quantize_chunk_fp8(
+        ctypes.byref(p), _ptr(q_cur, "q_cur", dt, n["act_cur"]),
+        _ptr(k_cur, "k_cur", dt, n["act_cur"]), _ptr(v_cur, "v_cur", dt, n["act_cur"]),
+        ctypes.byref(fp), _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
+    _check(st, "fkv_quantize_chunk_fp8")
+
+
+def attend_compressed_fp8(p: Params, cache, kept_cnt, out, ws, stream=None):
+    """Step 5 over the e4m3 cache (fkv_attend_compressed_fp8), bf16 out."""
+    n, dt = _shapes(p), _act_dtype(p)
+    fp = make_fp8_cache(p, cache)
+    st = _lib.load().fkv_attend_compressed_fp8(
+        ctypes.byref(p), ctypes.byref(fp), _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]),
+        _ptr(out, "out", dt, n["act_cur"]), _ptr(ws, "ws", torch.uint8, n["ws"]), _stream(stream))
+    _check(st, "fkv_attend_compressed_fp8")
+
+
 def read_status(ws: torch.Tensor, stream=None):
     """(first device-side status since init, (layer*H + head) it was seen on or -1).
     Synchronises the stream."""

@@ -50,6 +50,18 @@ class StepIO(ctypes.Structure):
     _fields_ = [(n, c_vp) for n in STEP_IO_FIELDS]
 
 
+FP8_CACHE_FIELDS = (
+    "k_comp", "v_comp", "k_comp_scale", "v_comp_scale", "k_cur", "v_cur", "k_cur_scale",
+    "v_cur_scale", "q_cur", "q_scale",
+)
+
+
+class Fp8Cache(ctypes.Structure):
+    """fkv_fp8_cache_t."""
+
+    _fields_ = [(n, c_vp) for n in FP8_CACHE_FIELDS]
+
+
 # name -> (restype, argtypes), exactly the declarations of include/fkv.h
 SIGNATURES = {
     "fkv_status_string": (ctypes.c_char_p, [c_i32]),
@@ -71,6 +83,12 @@ SIGNATURES = {
     "fkv_compact_gather_rope": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "fkv_cache_advance": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp]),
     "fkv_step": (c_i32, [ctypes.POINTER(Params), ctypes.POINTER(StepIO), c_vp, c_vp]),
+    "fkv_compact_gather_fp8": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp,
+                                       ctypes.POINTER(Fp8Cache), c_vp, c_vp]),
+    "fkv_quantize_chunk_fp8": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp,
+                                       ctypes.POINTER(Fp8Cache), c_vp, c_vp]),
+    "fkv_attend_compressed_fp8": (c_i32, [ctypes.POINTER(Params), ctypes.POINTER(Fp8Cache), c_vp,
+                                          c_vp, c_vp, c_vp]),
 }
 
 _lib = None

@@ -417,4 +417,78 @@ int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void*
                    io->out, ws, s);
 }
 
+
+// ---- FP8 compressed cache ------------------------------------------------------
+static bool fp8_supported(const Dims& d) {
+  return d.bf16 && !d.token && !d.static_token_mask && d.D == 128;
+}
+static bool aligned4(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; }
+
+int32_t fkv_compact_gather_fp8(const fkv_params_t* p, const void* k_hist, const void* v_hist,
+                               const int32_t* kept_idx, const int32_t* kept_cnt,
+                               const fkv_fp8_cache_t* c, void* ws, void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (!fp8_supported(d)) return FKV_ERR_UNSUPPORTED;
+  if (!c || ((!k_hist || !v_hist) && d.N > 0) || (!kept_idx && d.max_kept > 0) || !kept_cnt)
+    return FKV_ERR_INVALID_ARG;
+  if (((!c->k_comp || !c->v_comp) && d.comp_rows > 0) ||
+      ((!c->k_comp_scale || !c->v_comp_scale) && d.F > 0))
+    return FKV_ERR_INVALID_ARG;
+  if (!aligned16(k_hist) || !aligned16(v_hist) || !aligned16(c->k_comp) ||
+      !aligned16(c->v_comp) || !aligned4(c->k_comp_scale) || !aligned4(c->v_comp_scale))
+    return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  if (d.F == 0) return FKV_OK;  // nothing can be kept
+  return cuda_status(launch_quant_segments(
+      d, int(d.max_kept), d.N, d.comp_rows, kept_idx, kept_cnt, k_hist, v_hist, c->k_comp,
+      c->v_comp, c->k_comp_scale, c->v_comp_scale, status_ptr(ws),
+      static_cast<cudaStream_t>(stream)));
+}
+
+int32_t fkv_quantize_chunk_fp8(const fkv_params_t* p, const void* q_cur, const void* k_cur,
+                               const void* v_cur, const fkv_fp8_cache_t* c, void* ws,
+                               void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (!fp8_supported(d)) return FKV_ERR_UNSUPPORTED;
+  if (!c || !q_cur || !k_cur || !v_cur || !c->q_cur || !c->q_scale || !c->k_cur || !c->v_cur ||
+      !c->k_cur_scale || !c->v_cur_scale)
+    return FKV_ERR_INVALID_ARG;
+  if (!aligned16(q_cur) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(c->q_cur) ||
+      !aligned16(c->k_cur) || !aligned16(c->v_cur) || !aligned4(c->q_scale) ||
+      !aligned4(c->k_cur_scale) || !aligned4(c->v_cur_scale))
+    return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = cuda_status(launch_quant_segments(d, d.Fc, d.Lq, d.Lq, nullptr, nullptr, k_cur, v_cur,
+                                              c->k_cur, c->v_cur, c->k_cur_scale,
+                                              c->v_cur_scale, status_ptr(ws), s))))
+    return st;
+  return cuda_status(launch_quant_rows(d, q_cur, c->q_cur, c->q_scale, s));
+}
+
+int32_t fkv_attend_compressed_fp8(const fkv_params_t* p, const fkv_fp8_cache_t* c,
+                                  const int32_t* kept_cnt, void* out, void* ws, void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (!fp8_supported(d) || d.T < 128) return FKV_ERR_UNSUPPORTED;
+  if (!c || !kept_cnt || !out || !c->q_cur || !c->q_scale || !c->k_cur || !c->v_cur ||
+      !c->k_cur_scale || !c->v_cur_scale)
+    return FKV_ERR_INVALID_ARG;
+  if (((!c->k_comp || !c->v_comp) && d.comp_rows > 0) ||
+      ((!c->k_comp_scale || !c->v_comp_scale) && d.F > 0))
+    return FKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {c->q_cur, c->k_cur, c->v_cur, c->k_comp, c->v_comp, out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  if (d.LH == 0 || d.Lq == 0) return FKV_OK;
+  return cuda_status(launch_attend_fp8_sm100(d, *c, kept_cnt, out, status_ptr(ws),
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

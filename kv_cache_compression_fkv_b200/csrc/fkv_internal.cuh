@@ -109,8 +109,21 @@ cudaError_t launch_advance(const Dims& d, int64_t out_segments, const void* k_co
                            const void* v_cur, void* k_next, void* v_next, int32_t* status,
                            cudaStream_t s);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
+cudaError_t launch_quant_segments(const Dims& d, int n_slots, int64_t src_rows, int64_t dst_rows,
+                                  const int32_t* kept_idx, const int32_t* kept_cnt,
+                                  const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                                  float* scale_k, float* scale_v, int32_t* status,
+                                  cudaStream_t s);
+cudaError_t launch_quant_rows(const Dims& d, const void* src, void* dst, float* scales,
+                              cudaStream_t s);
+cudaError_t launch_attend_fp8_sm100(const Dims& d, const fkv_fp8_cache_t& c,
+                                    const int32_t* kept_cnt, void* out, int32_t* status,
+                                    cudaStream_t s);
 cudaError_t launch_attend_simt(const Dims& d, const void* q_cur, const void* k_cur,
                                const void* v_cur, const void* k_comp, const void* v_comp,
                                const int32_t* kept_cnt, void* out, cudaStream_t s);
+
+// SM count of the current device (cached per device; 148 if unknown).
+int num_sms();
 
 }  // namespace fkv

@@ -314,5 +314,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // 128-byte swizzle, out-of-range rows read as zero.  Returns false on error.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t slabs,
                     uint64_t row_stride_bytes, uint64_t slab_stride_bytes);
+// Host: the same for 1-byte elements (e4m3 codes): [slabs][rows][128] bytes,
+// box [1][128][128], one 128-byte swizzle atom per row.
+bool make_tmap_u8(CUtensorMap* map, const void* base, uint64_t rows, uint64_t slabs,
+                  uint64_t row_stride_bytes, uint64_t slab_stride_bytes);
 
 }  // namespace fkv

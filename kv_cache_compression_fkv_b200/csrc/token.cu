@@ -138,7 +138,6 @@ __global__ void phi_generic_kernel(int D, int64_t N, int64_t S, int64_t n_c,
   }
 }
 
-int num_sms();
 
 cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
                                float* qbar, float* seg_score, cudaStream_t s) {

@@ -52,8 +52,52 @@ def test_struct_layout_matches_header(tmp_path, lib):
     assert got == [ctypes.sizeof(P), P.scale.offset, P.granularity.offset, ctypes.sizeof(S), S.out.offset]
 
 
+def test_fp8_cache_layout_matches_header(tmp_path, lib):
+    fields = _lib.FP8_CACHE_FIELDS
+    prog = tmp_path / "layout8.c"
+    body = " ".join(f'printf("%zu ", offsetof(fkv_fp8_cache_t, {f}));' for f in fields)
+    prog.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "fkv.h"\n'
+                    "int main(void){" + body + ' printf("%zu\\n", sizeof(fkv_fp8_cache_t)); return 0;}\n')
+    exe = tmp_path / "layout8"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(prog), "-o", str(exe)], check=True)
+    got = list(map(int, subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()))
+    C = _lib.Fp8Cache
+    assert got == [getattr(C, f).offset for f in fields] + [ctypes.sizeof(C)]
+
+
+def _fp8_params(**kw):
+    base = dict(L=1, H=2, D=128, T=128, F=4, Fc=1, dtype="bf16", comp_rows=4 * 128, score_stride=1)
+    base.update(kw)
+    return fkv.make_params(**base)
+
+
+def test_fp8_entry_points_validate_before_launch(lib):
+    p = _fp8_params()
+    c = _lib.Fp8Cache()
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails first
+    bp = ctypes.byref(p)
+    # null cache struct / null members
+    assert lib.fkv_compact_gather_fp8(bp, fake, fake, fake, fake, None, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_compact_gather_fp8(bp, fake, fake, fake, fake, ctypes.byref(c), fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_quantize_chunk_fp8(bp, fake, fake, fake, ctypes.byref(c), fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_attend_compressed_fp8(bp, ctypes.byref(c), fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    # unsupported configurations
+    for bad in (_fp8_params(dtype="fp32", D=64), _fp8_params(granularity="token", n_score_q=4, sink_tokens=128,
+                                                              recent_tokens=128)):
+        assert lib.fkv_quantize_chunk_fp8(ctypes.byref(bad), fake, fake, fake, ctypes.byref(c), fake,
+                                          None) == _lib.FKV_ERR_UNSUPPORTED
+    small_t = _fp8_params(T=64, comp_rows=4 * 64)
+    assert lib.fkv_attend_compressed_fp8(ctypes.byref(small_t), ctypes.byref(c), fake, fake, fake,
+                                         None) == _lib.FKV_ERR_UNSUPPORTED
+    # misaligned code buffer
+    for f in _lib.FP8_CACHE_FIELDS:
+        setattr(c, f, 1 << 20)
+    c.k_comp = (1 << 20) + 8
+    assert lib.fkv_compact_gather_fp8(bp, fake, fake, fake, fake, ctypes.byref(c), fake, None) == _lib.FKV_ERR_INVALID_ARG
+
+
 def test_status_strings_and_version(lib):
-    assert lib.fkv_abi_version() == 2
+    assert lib.fkv_abi_version() == 3
     for code in range(8):
         assert lib.fkv_status_string(code).decode().startswith("FKV_")
     assert lib.fkv_status_string(99) == b"FKV_ERR_UNKNOWN"

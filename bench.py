@@ -268,6 +268,39 @@ def run_ours(args, rank, world, local_rank):
     part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
             for j, n in enumerate(["score", "select", "gather", "attend", "gather_rope"])}
 
+    # ---- FP8 (e4m3) compressed cache: the same scoring and selection, then the
+    # e4m3 compaction, the chunk's quantisation and the kind::f8f6f4 attention
+    fp8 = None
+    if (w.granularity == "frame" and not w.static_token_mask and w.dtype == "bf16" and w.D == 128
+            and w.T >= 128):
+        c8 = fkv.allocate_fp8(p, dev)
+        out8 = torch.empty_like(outs["out"])
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            flush.fill_(i & 0xFF)
+            e = fev[i - args.warmup] if i >= args.warmup else None
+            if e: e[0].record(stream)  # noqa: E701
+            fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
+                               outs["seg_score"], outs["ws"], k_cur=x["k_cur"])
+            if e: e[1].record(stream)  # noqa: E701
+            fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
+                            x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])
+            if e: e[2].record(stream)  # noqa: E701
+            fkv.compact_gather_fp8(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
+                                   c8, outs["ws"])
+            if e: e[3].record(stream)  # noqa: E701
+            fkv.quantize_chunk_fp8(p, x["q_cur"], x["k_cur"], x["v_cur"], c8, outs["ws"])
+            if e: e[4].record(stream)  # noqa: E701
+            fkv.attend_compressed_fp8(p, c8, outs["kept_cnt"], out8, outs["ws"])
+            if e: e[5].record(stream)  # noqa: E701
+        torch.cuda.synchronize(dev)
+        st, det = fkv.read_status(outs["ws"])
+        if st != 0:
+            raise RuntimeError(f"device status {st} on head {det} (fp8 path)")
+        fp8 = {n: statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(args.steps))
+               for j, n in enumerate(["score", "select", "gather", "quant", "attend"])}
+        fp8["step"] = statistics.mean(fev[i][0].elapsed_time(fev[i][5]) for i in range(args.steps))
+
     # ---- e2e: host buffers in, result out, through the same call.  Every step
     # copies its inputs from pinned host memory (H2D stream), runs fkv_step
     # (compute stream) and reads its result back (D2H stream); two buffer sets
@@ -421,6 +454,30 @@ def run_ours(args, rank, world, local_rank):
     }
     if lifecycle is not None:
         line["lifecycle"] = lifecycle
+    if fp8 is not None:
+        fp8_peak = 2.0 * peaks["bf16_tflops"]  # dense e4m3 = 2 x bf16 (nominal ratio)
+        kept_rows = float((outs["kept_cnt"].cpu().to(torch.int64) * w.T).sum())
+        g8_bytes = kept_rows * w.D * 3 * 2          # K and V: 2 B read, 1 B written per element
+        q8_bytes = float(w.L * w.H * w.Lq * w.D * 3 * 3)  # Q, K, V of the chunk
+        a8_tfs = alg["attn_flops"] / (fp8["attend"] * 1e-3) / 1e12
+        line["fp8"] = {
+            "ms_per_step": round(fp8["step"], 4),
+            "value_per_gpu": round(aggregate_throughput(w.L, 1, fp8["step"]), 3), "unit": UNIT,
+            "kernels": {
+                "compact_gather_fp8": {"ms": round(fp8["gather"], 4),
+                                       "GB/s": round(g8_bytes / (fp8["gather"] * 1e-3) / 1e9, 1),
+                                       "frac_hbm": round(g8_bytes / (fp8["gather"] * 1e-3) / 1e9
+                                                         / peaks["hbm_gbs"], 4)},
+                "quantize_chunk_fp8": {"ms": round(fp8["quant"], 4),
+                                       "GB/s": round(q8_bytes / (fp8["quant"] * 1e-3) / 1e9, 1),
+                                       "frac_hbm": round(q8_bytes / (fp8["quant"] * 1e-3) / 1e9
+                                                         / peaks["hbm_gbs"], 4)},
+                "attend_compressed_fp8": {"ms": round(fp8["attend"], 4), "TFLOP/s": round(a8_tfs, 2),
+                                          "peak": round(fp8_peak, 1),
+                                          "peak_kind": f"2 x {peak_kind} burst bf16",
+                                          "frac_tensor": round(a8_tfs / fp8_peak, 4)},
+            },
+        }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget)
     if dist is not None:

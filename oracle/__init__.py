@@ -14,6 +14,8 @@ Modules
   fkv_fp8     the e4m3 compressed cache: codes and per-segment scales (fp32
               decisions, as the kernels take them), dequantisation, and the
               error model of an fp8 tensor-core attention.
+  fkv_heuristics  the comparison selectors (uniform eviction, random drop
+              with a Philox4x64-10 priority per segment).
 
 Sources (page title and section):
   Forcing-KV (ai-feeds.com/i/paper/2605.09681): "关键模块" items 2 (static

@@ -53,8 +53,9 @@
 extern "C" {
 #endif
 
-/* 3: adds fkv_fp8_cache_t and the three *_fp8 entry points. */
-#define FKV_ABI_VERSION 3
+/* 3: adds fkv_fp8_cache_t and the three *_fp8 entry points;
+ * 4: adds fkv_select_heuristic. */
+#define FKV_ABI_VERSION 4
 
 typedef enum fkv_status {
   FKV_OK = 0,
@@ -295,6 +296,33 @@ int32_t fkv_cache_advance(const fkv_params_t* p, const void* k_comp, const void*
 /* Steps 1-5 in one call: score (dynamic / token heads), select, compact,
  * attend, all enqueued on `stream` in that order. */
 int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void* stream);
+
+/* ---- Comparison selectors --------------------------------------------------
+ * Forcing-KV (ai-feeds.com/i/paper/2605.09681, "与基线对比及工程启示", first
+ * item) measures itself against uniform eviction and random dropping at the
+ * same compression ratio; the pages define neither.  Reading: every head keeps
+ * its budget k_per_head[l][h] (k frames in frame mode, C candidate tokens in
+ * token mode) whatever its role, and the output has the format of
+ * fkv_select_topk (kept_idx ascending, entries past kept_cnt untouched; token
+ * mode adds the sink [0, S) and recent [N-R, N) tokens).
+ *   FKV_POLICY_UNIFORM: of the n segments (frames, or candidates) keep
+ *     floor(i * n / k) for i < k; seg_score is not used (may be NULL).
+ *   FKV_POLICY_RANDOM: keep the k segments of largest priority, ties to the
+ *     lower index, where the priority of segment s of head lh is the first
+ *     64-bit word w of Philox4x64-10 (Salmon et al., "Parallel random
+ *     numbers: as easy as 1, 2, 3", SC 2011) at counter (s, lh, 0, 0) and
+ *     key (seed, 0), as (w >> 40) * 2^-24.  The priorities are written to
+ *     seg_score (float [L*H][nseg], device) and then ranked.
+ * Frame mode with FKV_FLAG_STATIC_TOKEN_MASK: FKV_ERR_UNSUPPORTED.  An unknown
+ * policy: FKV_ERR_INVALID_ARG.  k out of range: clamped, FKV_ERR_DEVICE_ARG. */
+typedef enum fkv_policy {
+  FKV_POLICY_UNIFORM = 0,
+  FKV_POLICY_RANDOM = 1
+} fkv_policy_t;
+
+int32_t fkv_select_heuristic(const fkv_params_t* p, int32_t policy, uint64_t seed,
+                             const int32_t* k_per_head, float* seg_score, int32_t* kept_idx,
+                             int32_t* kept_cnt, void* ws, void* stream);
 
 /* ---- FP8 (e4m3) compressed cache ------------------------------------------
  * Forcing-KV (ai-feeds.com/i/paper/2605.09681), "与现有产品/工作流的接口" item

@@ -227,6 +227,23 @@ def select_topk(p: Params, seg_score, head_role, static_mask, k_per_head, kept_i
     _check(st, "fkv_select_topk")
 
 
+def select_heuristic(p: Params, policy: str, seed: int, k_per_head, kept_idx, kept_cnt, ws,
+                     seg_score=None, stream=None):
+    """Comparison selector of every head (fkv_select_heuristic): policy
+    "uniform" (evenly spaced segments) or "random" (largest Philox4x64-10
+    priorities; written to seg_score, which is then required)."""
+    n = _shapes(p)
+    pol = {"uniform": _lib.FKV_POLICY_UNIFORM, "random": _lib.FKV_POLICY_RANDOM}[policy]
+    st = _lib.load().fkv_select_heuristic(
+        ctypes.byref(p), pol, int(seed) & ((1 << 64) - 1),
+        _ptr(k_per_head, "k_per_head", torch.int32, n["heads"]),
+        _ptr(seg_score, "seg_score", torch.float32, n["seg"], optional=policy == "uniform"),
+        _ptr(kept_idx, "kept_idx", torch.int32, n["kept"]),
+        _ptr(kept_cnt, "kept_cnt", torch.int32, n["heads"]), _ptr(ws, "ws", torch.uint8, n["ws"]),
+        _stream(stream))
+    _check(st, "fkv_select_heuristic")
+
+
 def compact_gather(p: Params, k_hist, v_hist, kept_idx, kept_cnt, k_comp, v_comp, ws, stream=None):
     n, dt = _shapes(p), _act_dtype(p)
     st = _lib.load().fkv_compact_gather(

@@ -22,6 +22,8 @@ FKV_GRAN_FRAME = 0
 FKV_GRAN_TOKEN = 1
 FKV_FLAG_SCORE_WITH_CHUNK = 1
 FKV_FLAG_STATIC_TOKEN_MASK = 2
+FKV_POLICY_UNIFORM = 0
+FKV_POLICY_RANDOM = 1
 
 c_i32, c_i64, c_f32, c_vp, c_sz = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
 
@@ -83,6 +85,8 @@ SIGNATURES = {
     "fkv_compact_gather_rope": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "fkv_cache_advance": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp]),
     "fkv_step": (c_i32, [ctypes.POINTER(Params), ctypes.POINTER(StepIO), c_vp, c_vp]),
+    "fkv_select_heuristic": (c_i32, [ctypes.POINTER(Params), c_i32, ctypes.c_uint64, c_vp, c_vp, c_vp,
+                                     c_vp, c_vp, c_vp]),
     "fkv_compact_gather_fp8": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp,
                                        ctypes.POINTER(Fp8Cache), c_vp, c_vp]),
     "fkv_quantize_chunk_fp8": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp,

@@ -418,6 +418,23 @@ int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void*
 }
 
 
+// ---- comparison selectors -------------------------------------------------------
+int32_t fkv_select_heuristic(const fkv_params_t* p, int32_t policy, uint64_t seed,
+                             const int32_t* k_per_head, float* seg_score, int32_t* kept_idx,
+                             int32_t* kept_cnt, void* ws, void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (policy != FKV_POLICY_UNIFORM && policy != FKV_POLICY_RANDOM) return FKV_ERR_INVALID_ARG;
+  if (!d.token && d.static_token_mask) return FKV_ERR_UNSUPPORTED;
+  if (!k_per_head || !kept_cnt || (!kept_idx && d.max_kept > 0) ||
+      (policy == FKV_POLICY_RANDOM && !seg_score && d.nseg > 0))
+    return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  return cuda_status(launch_heuristic(d, policy, seed, k_per_head, seg_score, kept_idx, kept_cnt,
+                                      status_ptr(ws), static_cast<cudaStream_t>(stream)));
+}
+
 // ---- FP8 compressed cache ------------------------------------------------------
 static bool fp8_supported(const Dims& d) {
   return d.bf16 && !d.token && !d.static_token_mask && d.D == 128;

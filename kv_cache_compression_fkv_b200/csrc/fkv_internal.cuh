@@ -119,6 +119,10 @@ cudaError_t launch_quant_rows(const Dims& d, const void* src, void* dst, float* 
 cudaError_t launch_attend_fp8_sm100(const Dims& d, const fkv_fp8_cache_t& c,
                                     const int32_t* kept_cnt, void* out, int32_t* status,
                                     cudaStream_t s);
+// Comparison selectors (uniform eviction / random drop) of every head.
+cudaError_t launch_heuristic(const Dims& d, int32_t policy, uint64_t seed,
+                             const int32_t* k_per_head, float* seg_score, int32_t* kept_idx,
+                             int32_t* kept_cnt, int32_t* status, cudaStream_t s);
 cudaError_t launch_attend_simt(const Dims& d, const void* q_cur, const void* k_cur,
                                const void* v_cur, const void* k_comp, const void* v_comp,
                                const int32_t* kept_cnt, void* out, cudaStream_t s);

@@ -27,7 +27,7 @@ __global__ void select_frame_kernel(int F, const float* __restrict__ seg_score,
   __shared__ int warp_counts[32];
   const int lh = blockIdx.x;
   const int f = threadIdx.x;
-  const bool dyn = head_role[lh] != 0;
+  const bool dyn = head_role ? head_role[lh] != 0 : true;  // no roles: every head ranked
   int k = 0;
   if (dyn) {
     k = k_per_head[lh];

@@ -97,7 +97,7 @@ def test_fp8_entry_points_validate_before_launch(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fkv_abi_version() == 3
+    assert lib.fkv_abi_version() == 4
     for code in range(8):
         assert lib.fkv_status_string(code).decode().startswith("FKV_")
     assert lib.fkv_status_string(99) == b"FKV_ERR_UNKNOWN"
@@ -168,3 +168,18 @@ def test_null_and_misaligned_pointers_fail_before_launch(lib):
     assert lib.fkv_step(ctypes.byref(bad), ctypes.byref(io), fake, None) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_workspace_init(fake + 8, 512, None) == _lib.FKV_ERR_WORKSPACE
     assert lib.fkv_read_status(None, None, None, None) == _lib.FKV_ERR_WORKSPACE
+
+
+def test_heuristic_selector_validates_before_launch(lib):
+    p = _fp8_params()
+    fake = ctypes.c_void_p(1 << 20)
+    bp = ctypes.byref(p)
+    assert lib.fkv_select_heuristic(bp, 7, 1, fake, fake, fake, fake, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    # random needs seg_score; uniform does not (but needs the kept arrays)
+    assert lib.fkv_select_heuristic(bp, _lib.FKV_POLICY_RANDOM, 1, fake, None, fake, fake, fake,
+                                    None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_select_heuristic(bp, _lib.FKV_POLICY_UNIFORM, 1, fake, None, None, fake, fake,
+                                    None) == _lib.FKV_ERR_INVALID_ARG
+    tm = _fp8_params(static_token_mask=True)
+    assert lib.fkv_select_heuristic(ctypes.byref(tm), _lib.FKV_POLICY_UNIFORM, 1, fake, None, fake,
+                                    fake, fake, None) == _lib.FKV_ERR_UNSUPPORTED

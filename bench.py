@@ -199,8 +199,16 @@ def run_ours(args, rank, world, local_rank):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local_rank)
-    w = replica_workload(wl.get(args.workload), rank, world)
-    x_cpu = wl.generate(w)
+    from kv_cache_compression_fkv_b200 import shard
+    base = wl.get(args.workload)
+    if args.split == "heads":
+        # strong scaling: rank r runs its contiguous range of the L*H heads of one step
+        h0, h1 = shard.head_range(base.L * base.H, world, rank)
+        x_cpu = shard.shard_inputs(wl.generate(base), h0, h1)
+        w = shard.local_workload(base, h0, h1)
+    else:
+        w = replica_workload(base, rank, world)
+        x_cpu = wl.generate(w)
     p = fkv.params_for(w)
     stream = torch.cuda.current_stream(dev)
     x = {k: v.to(dev) for k, v in x_cpu.items()}
@@ -398,11 +406,29 @@ def run_ours(args, rank, world, local_rank):
         if st != 0:
             raise RuntimeError(f"device status {st} on head {det}")
 
+    # heads split: the all-gather of O that gives every rank the whole output
+    gather_ms = None
+    if args.split == "heads" and dist is not None:
+        gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.warmup + args.steps):
+            if i >= args.warmup:
+                gev[i - args.warmup][0].record(stream)
+            shard.gather_heads(outs["out"], base.L * base.H, world)
+            if i >= args.warmup:
+                gev[i - args.warmup][1].record(stream)
+        torch.cuda.synchronize(dev)
+        gather_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in gev), dist, dev)
+
     alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
                       else torch.ones(w.L, w.H))
     peaks, peak_kind = load_peaks()
-    value = aggregate_throughput(w.L * args.steps, world, total_ms)
-    e2e_value = aggregate_throughput(w.L * args.steps, world, e2e_ms)
+    if args.split == "heads":  # all ranks together run one whole step per step
+        value = aggregate_throughput(base.L * args.steps, 1, total_ms)
+        e2e_value = aggregate_throughput(base.L * args.steps, 1, e2e_ms)
+    else:
+        value = aggregate_throughput(w.L * args.steps, world, total_ms)
+        e2e_value = aggregate_throughput(w.L * args.steps, world, e2e_ms)
     attn_tfs = alg["attn_flops"] / (part["attend"] * 1e-3) / 1e12
     gather_gbs = alg["gather_bytes"] / (part["gather"] * 1e-3) / 1e9
     score_tfs = alg["score_flops"] / (part["score"] * 1e-3) / 1e12
@@ -438,12 +464,17 @@ def run_ours(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total_ms / args.steps, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if args.split == "heads" else "weak",
+        "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic (seeded, Wan-shaped)",
-        "config": {"workload": w.name, "L": w.L, "H": w.H, "D": w.D, "T": w.T, "F": w.F, "Fc": w.Fc,
-                   "granularity": w.granularity, "kept_per_head": int(outs["kept_cnt"][0, 0]),
+        "config": {"workload": base.name, "L": base.L, "H": base.H, "D": w.D, "T": w.T, "F": w.F,
+                   "Fc": w.Fc, "granularity": w.granularity,
+                   "kept_per_head": int(outs["kept_cnt"][0, 0]),
                    "l2": "flushed between timed steps (256 MiB write outside the events)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+                   "parallelism": (f"heads split over {world} GPUs" if args.split == "heads" and world > 1
+                                   else f"replicas x{world}" if world > 1 else "single GPU"),
+                   **({"heads_per_rank": f"{w.H} (rank {rank})", "gather_out_ms": round(gather_ms, 4)}
+                      if gather_ms is not None else {})},
         "impl": "ours",
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -564,6 +595,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="480p", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas per GPU (weak scaling) or the heads of "
+                         "one step split across GPUs (strong scaling)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -276,6 +276,20 @@ def run_ours(args, rank, world, local_rank):
     part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
             for j, n in enumerate(["score", "select", "gather", "attend", "gather_rope"])}
 
+    # comparison selectors (uniform eviction / random drop), same budgets
+    hev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        hev[i][0].record(stream)
+        fkv.select_heuristic(p, "uniform", 1, x["k_per_head"], outs["kept_idx"], outs["kept_cnt"],
+                             outs["ws"])
+        hev[i][1].record(stream)
+        fkv.select_heuristic(p, "random", 1 + i, x["k_per_head"], outs["kept_idx"], outs["kept_cnt"],
+                             outs["ws"], seg_score=outs["seg_score"])
+        hev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    heur = {n: statistics.mean(hev[i][j].elapsed_time(hev[i][j + 1]) for i in range(args.steps))
+            for j, n in enumerate(["uniform", "random"])}
+
     # ---- FP8 (e4m3) compressed cache: the same scoring and selection, then the
     # e4m3 compaction, the chunk's quantisation and the kind::f8f6f4 attention
     fp8 = None
@@ -447,6 +461,8 @@ def run_ours(args, rank, world, local_rank):
                            "frac_tensor": round(score_tfs / peaks["bf16_tflops"], 4),
                            "frac_hbm": round(score_gbs / peaks["hbm_gbs"], 4)},
         "select_topk": {"ms": round(part["select"], 4)},
+        "select_heuristic": {"uniform_ms": round(heur["uniform"], 4),
+                             "random_ms": round(heur["random"], 4)},
         "compact_gather_rope": ({"ms": round(part["gather_rope"], 4),
                                  "GB/s": round(alg["gather_bytes"] / (part["gather_rope"] * 1e-3) / 1e9, 1),
                                  "frac_hbm": round(alg["gather_bytes"] / (part["gather_rope"] * 1e-3) / 1e9
@@ -506,7 +522,10 @@ def run_ours(args, rank, world, local_rank):
                 "attend_compressed_fp8": {"ms": round(fp8["attend"], 4), "TFLOP/s": round(a8_tfs, 2),
                                           "peak": round(fp8_peak, 1),
                                           "peak_kind": f"2 x {peak_kind} burst bf16",
-                                          "frac_tensor": round(a8_tfs / fp8_peak, 4)},
+                                          "frac_tensor": round(a8_tfs / fp8_peak, 4),
+                                          "traffic": committed_traffic(
+                                              "attend_fp8", w.name,
+                                              kernel_source_hash(_attend_fp8_sources()))},
             },
         }
     if rank == 0 and not args.no_cpu_baseline and world == 1:
@@ -519,7 +538,12 @@ def run_ours(args, rank, world, local_rank):
 
 def _attend_sources():
     """Source files of the attention kernel (the traffic record is void once they change)."""
-    return ["attend_sm100.cu", "sm100_common.cuh"]
+    return ["attend_sm100.cu", "attend_common.cuh", "sm100_common.cuh"]
+
+
+def _attend_fp8_sources():
+    """Source files of the e4m3 attention kernel."""
+    return ["attend_fp8_sm100.cu", "attend_common.cuh", "sm100_common.cuh"]
 
 
 # --------------------------------------------------------------------------- CPU oracle

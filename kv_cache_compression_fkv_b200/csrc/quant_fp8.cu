@@ -25,6 +25,7 @@ namespace fkv {
 
 constexpr int kSegCta = 8;         // CTAs per segment (one cluster)
 constexpr int kSegThreads = 256;
+constexpr int kSegBatch = 4;       // loads in flight per thread
 constexpr int kRowThreads = 256;   // 16 rows of 16 lanes per CTA pass
 
 __device__ __forceinline__ float amax8(uint4 raw) {
@@ -104,8 +105,18 @@ quant_segments_kernel(int32_t T_, int32_t vpr, int32_t n_slots, int32_t F, int64
   uint2* dst = (is_v ? dst_v : dst_k) + (int64_t(lh) * dst_rows + int64_t(slot) * T_) * vpr;
   const int64_t v0 = nvec * rank / kSegCta, v1 = nvec * (rank + 1) / kSegCta;
 
+  // kSegBatch independent 16-byte loads in flight per thread in both passes
   float m = 0.f;
-  for (int64_t i = v0 + threadIdx.x; i < v1; i += kSegThreads) m = fmaxf(m, amax8(__ldg(src + i)));
+  for (int64_t b = v0 + threadIdx.x; b < v1; b += kSegThreads * kSegBatch) {
+    uint4 r[kSegBatch];
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) {
+      const int64_t i = b + int64_t(u) * kSegThreads;
+      r[u] = i < v1 ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) m = fmaxf(m, amax8(r[u]));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = m;
@@ -123,8 +134,19 @@ quant_segments_kernel(int32_t T_, int32_t vpr, int32_t n_slots, int32_t F, int64
   scale_pair(amax, &scale, &inv);
   if (rank == 0 && threadIdx.x == 0)
     (is_v ? scale_v : scale_k)[int64_t(lh) * n_slots + slot] = scale;
-  for (int64_t i = v0 + threadIdx.x; i < v1; i += kSegThreads)
-    __stcs(dst + i, quant8(__ldcs(src + i), inv));
+  for (int64_t b = v0 + threadIdx.x; b < v1; b += kSegThreads * kSegBatch) {
+    uint4 r[kSegBatch];
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) {
+      const int64_t i = b + int64_t(u) * kSegThreads;
+      if (i < v1) r[u] = __ldcs(src + i);
+    }
+#pragma unroll
+    for (int u = 0; u < kSegBatch; ++u) {
+      const int64_t i = b + int64_t(u) * kSegThreads;
+      if (i < v1) __stcs(dst + i, quant8(r[u], inv));
+    }
+  }
   cluster.sync();  // no CTA leaves while another may still read its s_amax
 }
 

@@ -1,5 +1,6 @@
 """Compaction with temporal RoPE re-positioning of the kept keys, against the
-oracle (fp64 rotation of the same inputs, rounded once by the GPU)."""
+oracle (fp64 rotation of the same inputs, rounded once by the GPU).  The kept
+lists come from a seeded host generator, the same for both sides."""
 import numpy as np
 import pytest
 import torch
@@ -19,10 +20,11 @@ def test_compact_gather_rope(cuda_device, dtype, n_pairs):
                   static_frames=(0, 3, 6), k_dynamic=3, score_stride=2, dtype=dtype, seed=61,
                   style="video")
     x = wl.generate(w)
-    p = fkv.params_for(w)
+    p = fkv.params_for(w, comp_rows=w.F * w.T)  # room for every frame: the lists are random
     d = parity.upload(x)
     o = fkv.allocate(p)
-    fkv.step(p, d, o)
+    # seeded kept lists from the host, the same for both sides
+    o["kept_idx"], o["kept_cnt"] = (t.cuda() for t in wl.random_kept(w, seed=62))
     omega = torch.tensor(10000.0 ** (-np.arange(n_pairs) / max(n_pairs, 1)), dtype=torch.float32)
     kc = torch.full_like(o["k_comp"], float("nan"))
     vc = torch.full_like(o["v_comp"], float("nan"))

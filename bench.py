@@ -43,6 +43,9 @@ import fkv_workloads as wl  # noqa: E402
 METRIC = "fkv_step chunk-steps/s per layer"
 UNIT = "chunk-steps/s per layer"
 SPEC_BF16_TFLOPS = 2250.0
+# MUFU exp2 rate derived from unit counts and clocks: 16 per SM per cycle,
+# 148 SMs, 1965 MHz maximum SM clock.
+SFU_EXP2_PER_S = 16 * 148 * 1965e6
 SPEC_HBM_GBS = 7700.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -80,8 +83,15 @@ def algorithmic(w, kept_cnt, head_role):
         n_c = w.N - w.sink_tokens - w.recent_tokens
         score_flops = 2.0 * n_c * w.D * w.L * w.H
         score_bytes = float(w.L * w.H * (n_c + w.n_score_q) * w.D * elem)
+    # exponentials the scoring must evaluate: every logit of every scoring row
+    # (frame mode; the chunk's own keys too when they join the normaliser)
+    if w.granularity == "frame":
+        keys_scored = w.N + (w.Lq if w.score_with_chunk else 0)
+        score_exps = float(n_dyn * n_s * keys_scored)
+    else:
+        score_exps = 0.0
     return {"attn_flops": attn_flops, "gather_bytes": gather_bytes,
-            "score_flops": score_flops, "score_bytes": score_bytes}
+            "score_flops": score_flops, "score_bytes": score_bytes, "score_exps": score_exps}
 
 
 # --------------------------------------------------------------------------- clocks
@@ -458,6 +468,10 @@ def run_ours(args, rank, world, local_rank):
     kernels = {
         "score_segments": {"ms": round(part["score"], 4), "TFLOP/s": round(score_tfs, 2),
                            "GB/s": round(score_gbs, 1),
+                           **({"bound": "sfu", "exp2_per_s": round(alg["score_exps"] / (part["score"] * 1e-3), 1),
+                               "peak_exp2_per_s": SFU_EXP2_PER_S,
+                               "frac_sfu": round(alg["score_exps"] / (part["score"] * 1e-3) / SFU_EXP2_PER_S, 4)}
+                              if alg["score_exps"] else {}),
                            "frac_tensor": round(score_tfs / peaks["bf16_tflops"], 4),
                            "frac_hbm": round(score_gbs / peaks["hbm_gbs"], 4)},
         "select_topk": {"ms": round(part["select"], 4)},

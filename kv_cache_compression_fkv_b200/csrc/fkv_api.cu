@@ -173,7 +173,7 @@ static int32_t do_attend(const Dims& d, const void* q_cur, const void* k_cur, co
 static int32_t step_launch_count(const Dims& d) {
   int32_t n = 0;
   if (d.token) n += d.nseg > 0 ? 2 : 0;   // q-sum, phi
-  else n += d.F > 0 ? 2 : 0;              // partial statistics, finalize
+  else n += d.F > 0 ? 3 : 0;              // partial statistics, row merge, frame masses
   n += 1;                                 // select
   n += 1;                                 // gather
   n += 1;                                 // attention

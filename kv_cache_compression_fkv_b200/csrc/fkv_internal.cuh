@@ -73,9 +73,11 @@ cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void
                                     const void* k_cur, const uint8_t* head_role, float2* part_ml,
                                     cudaStream_t s);
 // part_ml holds, per head, F*split sub-segment entries followed (when
-// d.score_with_chunk) by one entry for the chunk's keys, each n_s rows.
+// d.score_with_chunk) by one entry for the chunk's keys, each n_s rows; the
+// finalize overwrites the m of each frame's first entry with that frame's
+// per-row mass.
 cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
-                                        const float2* part_ml, float2* row_ml, float* seg_score,
+                                        float2* part_ml, float2* row_ml, float* seg_score,
                                         cudaStream_t s);
 cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
                                float* qbar, float* seg_score, cudaStream_t s);

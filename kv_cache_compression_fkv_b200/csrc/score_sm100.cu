@@ -5,10 +5,10 @@
 //
 // A CTA owns (layer*head, 128 scoring queries, one half of a history frame):
 // the frame's T keys are cut into 128-key blocks that start at the frame's
-// first token, and the blocks are split into two sub-segments (first and
-// second half of the blocks), so equal frames are reduced in exactly the same
-// order (bit-equal statistics) while the grid has twice as many, shorter
-// CTAs.  For each query row i the CTA produces the sub-segment max
+// first token, and the blocks are split into kScoreSplit sub-segments of
+// consecutive blocks, so equal frames are reduced in exactly the same order
+// (bit-equal statistics) while the grid has kScoreSplit times as many,
+// shorter CTAs.  For each query row i the CTA produces the sub-segment max
 // m_{g,i} and sum l_{g,i} = sum_{j in g} 2^(z_ij - m_{g,i}) of the base-2
 // logits z = scale*log2(e)*q.k; score_finalize_kernel merges them per row and
 // sums the frame masses in a fixed order.
@@ -91,10 +91,14 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
     row0 = 0;
     nkeys = a.Lq;
   } else {
+    // sub-segment `sub` of frame f: its blocks [bs, be) of the frame's nbf,
+    // bs = ceil(sub * nbf / split) (equal frames are cut at the same blocks)
     const int f = g / kScoreSplit, sub = g - f * kScoreSplit;
-    const int nbh = ((a.T + 127) / 128 + 1) / 2;
-    row0 = f * a.T + (sub ? nbh * 128 : 0);
-    nkeys = sub ? a.T - nbh * 128 : (a.T < nbh * 128 ? a.T : nbh * 128);
+    const int nbf = (a.T + 127) / 128;
+    const int bs = (sub * nbf + kScoreSplit - 1) / kScoreSplit;
+    const int be = ((sub + 1) * nbf + kScoreSplit - 1) / kScoreSplit;
+    row0 = f * a.T + bs * 128;
+    nkeys = (be * 128 < a.T ? be * 128 : a.T) - bs * 128;
   }
   const int b0 = 0, b1 = nkeys > 0 ? (nkeys + 127) / 128 : 0;
   float2* out = a.part_ml + (int64_t(lh) * a.E + g) * a.n_s;

@@ -107,54 +107,87 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
 }
 
 // Frame masses from the partial statistics of G = F*split sub-segments per
-// head (split consecutive sub-segments per frame).  One CTA per (layer, head):
+// head (split consecutive sub-segments per frame, then the chunk's own entry
+// when it joins the normaliser):
 //   row merge   M_i = max_g m_{g,i},  L_i = sum_g l_{g,i} 2^(m_{g,i} - M_i)
 //               (stored as (M_i, 1/L_i) in row_ml),
-//   frame mass  mass_f = sum_i sum_{g in f} l_{g,i} 2^(m_{g,i} - M_i) / L_i,
-// each warp owning frames f = warp, warp + 8, ..., lanes striding the rows,
-// then a fixed shuffle tree: the order of every sum is fixed (deterministic).
+//   frame mass  mass_f = sum_i c_{f,i},  c_{f,i} = sum_{g in f} l_{g,i} 2^(m_{g,i} - M_i) / L_i.
+// Two kernels, every sum in a fixed order (deterministic, equal frames give
+// bit-equal masses):
+//   score_rows_kernel    one warp per (head, row): lanes stride the entries,
+//                        a fixed shuffle tree; c_{f,i} is written back over
+//                        the m of the frame's first sub-segment of the same
+//                        row (each warp touches only its own row);
+//   score_frames_kernel  one warp per (head, frame): lanes stride the rows,
+//                        a fixed shuffle tree.
+constexpr int kRowWarps = 8;
 constexpr int kFinThreads = 1024;
 
+__global__ void __launch_bounds__(kRowWarps * 32)
+score_rows_kernel(int F, int split, int with_chunk, int64_t n_s,
+                  const uint8_t* __restrict__ head_role, float2* __restrict__ part_ml,
+                  float2* __restrict__ row_ml) {
+  const int lh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t i = int64_t(blockIdx.x) * kRowWarps + warp;
+  if (!head_role[lh] || i >= n_s) return;  // warp-uniform
+  const int G = F * split + with_chunk;
+  const int E = F * split + 1;
+  float2* p = part_ml + int64_t(lh) * E * n_s + i;
+  float M = -INFINITY;
+  for (int g = lane; g < G; g += 32) M = fmaxf(M, p[int64_t(g) * n_s].x);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float Ls = 0.f;
+  for (int g = lane; g < G; g += 32) {
+    const float2 ml = p[int64_t(g) * n_s];
+    if (ml.y != 0.f) Ls += ml.y * exp2f(ml.x - M);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+  const float inv = 1.f / Ls;
+  if (lane == 0) row_ml[int64_t(lh) * n_s + i] = make_float2(M, inv);
+  float c[4];  // frames lane, lane + 32, ... (up to 128 frames per pass)
+  for (int f0 = 0; f0 < F; f0 += 128) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = f0 + lane + 32 * u;
+      c[u] = 0.f;
+      if (f < F) {
+        float t = 0.f;
+        for (int s2 = 0; s2 < split; ++s2) {
+          const float2 ml = p[int64_t(f * split + s2) * n_s];
+          if (ml.y != 0.f) t += ml.y * exp2f(ml.x - M);
+        }
+        c[u] = t * inv;
+      }
+    }
+    __syncwarp();  // every lane has read the entries this pass overwrites
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int f = f0 + lane + 32 * u;
+      if (f < F) p[int64_t(f * split) * n_s].x = c[u];
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kFinThreads)
-score_finalize_kernel(int F, int split, int with_chunk, int64_t n_s,
-                      const uint8_t* __restrict__ head_role, const float2* __restrict__ part_ml,
-                      float2* __restrict__ row_ml, float* __restrict__ seg_score) {
+score_frames_kernel(int F, int split, int64_t n_s, const uint8_t* __restrict__ head_role,
+                    const float2* __restrict__ part_ml, float* __restrict__ seg_score) {
   const int lh = blockIdx.x;
-  const int G = F * split + with_chunk;  // entries in the row normaliser
-  const int E = F * split + 1;           // entries per head in part_ml
+  const int E = F * split + 1;
   float* out = seg_score + int64_t(lh) * F;
   if (!head_role[lh]) {
     for (int f = threadIdx.x; f < F; f += blockDim.x) out[f] = 0.f;
     return;
   }
   const float2* p = part_ml + int64_t(lh) * E * n_s;
-  float2* rm = row_ml + int64_t(lh) * n_s;
-  for (int64_t i = threadIdx.x; i < n_s; i += blockDim.x) {
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int g = 0; g < G; ++g) M = fmaxf(M, p[int64_t(g) * n_s + i].x);
-    float Ls = 0.f;
-#pragma unroll 8
-    for (int g = 0; g < G; ++g) {
-      const float2 ml = p[int64_t(g) * n_s + i];
-      if (ml.y != 0.f) Ls += ml.y * exp2f(ml.x - M);
-    }
-    rm[i] = make_float2(M, 1.f / Ls);
-  }
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int f = warp; f < F; f += blockDim.x >> 5) {
+    const float2* cf = p + int64_t(f * split) * n_s;
     float acc = 0.f;
 #pragma unroll 4
-    for (int64_t i = lane; i < n_s; i += 32) {
-      const float2 MR = rm[i];
-      float t = 0.f;
-      for (int s = 0; s < split; ++s) {
-        const float2 ml = p[int64_t(f * split + s) * n_s + i];
-        if (ml.y != 0.f) t += ml.y * exp2f(ml.x - MR.x);
-      }
-      acc += t * MR.y;
-    }
+    for (int64_t i = lane; i < n_s; i += 32) acc += cf[i].x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) out[f] = acc;
@@ -181,10 +214,17 @@ cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void
 }
 
 cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
-                                        const float2* part_ml, float2* row_ml, float* seg_score,
+                                        float2* part_ml, float2* row_ml, float* seg_score,
                                         cudaStream_t s) {
-  score_finalize_kernel<<<d.LH, kFinThreads, 0, s>>>(d.F, split, d.score_with_chunk ? 1 : 0,
-                                                     d.n_s, head_role, part_ml, row_ml, seg_score);
+  if (d.n_s > 0) {
+    dim3 grid(unsigned((d.n_s + kRowWarps - 1) / kRowWarps), unsigned(d.LH));
+    score_rows_kernel<<<grid, kRowWarps * 32, 0, s>>>(d.F, split, d.score_with_chunk ? 1 : 0,
+                                                      d.n_s, head_role, part_ml, row_ml);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  score_frames_kernel<<<d.LH, kFinThreads, 0, s>>>(d.F, split, d.n_s, head_role, part_ml,
+                                                   seg_score);
   return cudaGetLastError();
 }
 

@@ -205,10 +205,10 @@ int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void*
  * deployment convenience of this library.
  *
  * Same arguments, results and host-side checks as fkv_score_segments.  The
- * scratch lives in a static 4 MiB device array inside the library (held by
+ * scratch lives in a static 16 MiB device array inside the library (held by
  * every GPU that loads the library until the process exits); sizes needing
- * more (fkv_workspace_size > 4 MiB, e.g. the 30-layer 480P batch) are
- * rejected with FKV_ERR_WORKSPACE and nothing is launched.  It calls no
+ * more (fkv_workspace_size > 16 MiB, e.g. the 1080P layer or the 30-layer
+ * 480P batch) are rejected with FKV_ERR_WORKSPACE and nothing is launched.  It calls no
  * cudaMalloc / cudaFree.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current) and caches it; make

@@ -17,7 +17,7 @@ WsLayout ws_layout(const Dims& d) {
   w.part_ml = w.row_ml = w.qbar = off;
   if (!d.token) {
     w.part_ml = off;
-    off = align256(off + sizeof(float2) * size_t(d.LH) * (size_t(d.F) * kScoreSplit + 1) *
+    off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(score_layout(d).E) *
                              size_t(d.n_s));
     w.row_ml = off;
     off = align256(off + sizeof(float2) * size_t(d.LH) * size_t(d.n_s));
@@ -136,7 +136,7 @@ static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, c
                          : launch_score_frame_simt(d, q_cur, k_hist, k_cur, head_role, part, s);
   if (e != cudaSuccess) return cuda_status(e);
   return cuda_status(
-      launch_score_frame_finalize(d, d.bf16 ? kScoreSplit : 1, head_role, part, rows, seg_score, s));
+      launch_score_frame_finalize(d, score_layout(d), head_role, part, rows, seg_score, s));
 }
 
 static int32_t do_select(const Dims& d, const float* seg_score, const uint8_t* head_role,

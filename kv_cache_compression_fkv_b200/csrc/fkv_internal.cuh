@@ -31,9 +31,31 @@ struct Dims {
   int elem;          // bytes per activation element
 };
 
-// Sub-segments per frame of the tensor-core scoring kernel (the CUDA-core
-// scoring produces one per frame).
-constexpr int kScoreSplit = 2;
+// Layout of the frame-mode partial softmax statistics (part_ml, float2
+// (max, sum), [head][scoring row][entry], a row's entries contiguous): per
+// head and row, F*split frame entries
+// (entry f*split + i is the i-th piece of frame f), then `chunk` entries for
+// the chunk's own keys when they join the normaliser; E entries per head.
+//   tensor-core scoring (bf16): one entry per 128-key block, split =
+//     ceil(T/128), chunk = ceil(Lq/128) or 0, E = F*split + chunk;
+//   CUDA-core scoring (fp32): one entry per frame, split = 1, chunk = 1 or 0,
+//     E = F + 1.
+struct ScoreLayout {
+  int split, chunk, E;
+};
+inline ScoreLayout score_layout(const Dims& d) {
+  ScoreLayout s;
+  if (d.bf16) {
+    s.split = (d.T + 127) / 128;
+    s.chunk = d.score_with_chunk ? int((d.Lq + 127) / 128) : 0;
+    s.E = d.F * s.split + s.chunk;
+  } else {
+    s.split = 1;
+    s.chunk = d.score_with_chunk ? 1 : 0;
+    s.E = d.F + 1;
+  }
+  return s;
+}
 
 // Workspace layout (byte offsets from the workspace base, 256-B aligned).
 struct WsLayout {
@@ -72,13 +94,12 @@ __device__ __forceinline__ uint32_t ordered_key(float x) {
 cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void* k_hist,
                                     const void* k_cur, const uint8_t* head_role, float2* part_ml,
                                     cudaStream_t s);
-// part_ml holds, per head, F*split sub-segment entries followed (when
-// d.score_with_chunk) by one entry for the chunk's keys, each n_s rows; the
+// part_ml has the layout of score_layout(d), [head][n_s rows][E entries]; the
 // finalize overwrites the m of each frame's first entry with that frame's
 // per-row mass.
-cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
-                                        float2* part_ml, float2* row_ml, float* seg_score,
-                                        cudaStream_t s);
+cudaError_t launch_score_frame_finalize(const Dims& d, const ScoreLayout& sl,
+                                        const uint8_t* head_role, float2* part_ml,
+                                        float2* row_ml, float* seg_score, cudaStream_t s);
 cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
                                float* qbar, float* seg_score, cudaStream_t s);
 cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uint8_t* head_role,

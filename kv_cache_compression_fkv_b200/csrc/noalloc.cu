@@ -23,10 +23,11 @@
 
 namespace fkv {
 
-// Scratch bound: covers the 480P and 1080P single-layer workloads (about
-// 0.5 MB and 1.3 MB of partial statistics) and any token-mode call with up to
-// 8192 (layer, head) pairs.
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+// Scratch bound: covers the 480P single-layer workload (about 6.6 MB of
+// per-block partial statistics) and any token-mode call with up to 32768
+// (layer, head) pairs; larger frame-mode calls (1080P, the 30-layer batch)
+// need a workspace.
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -1,25 +1,28 @@
-// Step 2 on the tensor cores: per-frame softmax statistics of the dynamic
+// Step 2 on the tensor cores: per-block softmax statistics of the dynamic
 // heads' scoring queries (Forcing-KV, ai-feeds.com/i/paper/2605.09681,
 // "关键模块" 3: history grouped by frame, each group scored by the current
 // queries' attention).
 //
-// A CTA owns (layer*head, 128 scoring queries, one half of a history frame):
-// the frame's T keys are cut into 128-key blocks that start at the frame's
-// first token, and the blocks are split into kScoreSplit sub-segments of
-// consecutive blocks, so equal frames are reduced in exactly the same order
-// (bit-equal statistics) while the grid has kScoreSplit times as many,
-// shorter CTAs.  For each query row i the CTA produces the sub-segment max
-// m_{g,i} and sum l_{g,i} = sum_{j in g} 2^(z_ij - m_{g,i}) of the base-2
-// logits z = scale*log2(e)*q.k; score_finalize_kernel merges them per row and
-// sums the frame masses in a fixed order.
+// Work unit = one 128-key block of one frame (blocks start at the frame's
+// first token; the last is ragged) -- or of the chunk's own keys when they join
+// the normaliser -- for one dynamic head and one tile of 128 scoring queries.
+// For each query row i the unit produces m_{b,i} = max_j z_ij and
+// l_{b,i} = sum_j 2^(z_ij - m_{b,i}) over the block's keys j, with base-2
+// logits z = scale*log2(e)*q.k, written as entry b of the head's partial
+// statistics; the finalize merges the entries per row and sums them per frame
+// in a fixed order.  Equal frames are therefore reduced in exactly the same
+// order (bit-equal masses) however the units are spread over CTAs.
 //
-// Warp roles (320 threads): warps 0-7 fold the logit tiles into (m, l), two
-// threads per query row (TMEM lane) with 64 columns each, merged at the end;
-// warp 8 issues the TMA loads (Q tile once; K blocks into a 2-stage ring,
-// 128-byte swizzle; the scoring rows q_cur[i*stride] come from a strided
-// tensor map); warp 9 issues S = Q K^T into a TMEM double buffer, so the MMAs
-// of the next block overlap the statistics of the current one.  96 KB of
-// shared memory and 256 TMEM columns let two CTAs share an SM.
+// The grid is persistent (two CTAs per SM): the dynamic heads are counted on
+// the device and CTA c takes units [c*U/G, (c+1)*U/G) of the U units, ordered
+// (dynamic head, query tile, block), so the work is balanced to one block and
+// the K pipeline runs on across units.  Warp roles (320 threads): warps 0-7
+// fold S into (m, l), two threads per query row (TMEM lane) with 64 columns
+// each, merged through a bounded mbarrier exchange; warp 8 issues the TMA
+// loads (the query tile when it changes; K blocks into a 2-stage ring, 128-byte
+// swizzle; the scoring rows q_cur[i*stride] come from a strided tensor map);
+// warp 9 issues S = Q K^T into a TMEM double buffer, so the MMAs of the next
+// block overlap the statistics of the current one.
 #include "fkv_internal.cuh"
 #include "sm100_common.cuh"
 
@@ -28,7 +31,7 @@ namespace sm100 {
 
 constexpr int kScoreStages = 2;
 constexpr int kScoreThreads = 320;
-constexpr int kScoreStatThreads = 256;
+constexpr int kScoreHalfThreads = 128;  // one column half of the statistics warps
 constexpr int kScoreProducerWarp = 8;
 constexpr int kScoreMmaWarp = 9;
 constexpr uint32_t kScoreIdesc = idesc_bf16(128, 128, false);
@@ -37,20 +40,23 @@ constexpr uint32_t kSOffK = kTileBytes;
 constexpr uint32_t kSOffBar = kSOffK + kScoreStages * kTileBytes;
 
 struct ScoreBars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[kScoreStages], k_empty[kScoreStages];
   uint64_t s_full[2], s_free[2];
+  uint64_t x_full[2], x_read[2];  // per S buffer: half 1 wrote (m, l) / half 0 read it
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
-  float2 xml[2][128];  // [column half][row] partial (max, sum) for the end merge
+  int n_dyn;
+  float2 xml[2][128];  // [S buffer][row] (m, l) of the second column half
 };
 
 constexpr size_t kScoreSmem = kSOffBar + sizeof(ScoreBars) + 1024;
 
 struct ScoreArgs {
-  int T, G, E;  // tokens per frame; history sub-segments (F * kScoreSplit); entries per head
-  int Lq, with_chunk;
+  int LH, T, F, nbf, nbc, E;  // blocks per frame / of the chunk (0: chunk not scored)
+  int n_qt;
+  int Lq;
   int64_t n_s;
   float sl2;
   const uint8_t* head_role;
@@ -76,37 +82,73 @@ __device__ __forceinline__ float2 merge_ml(float2 a, float2 b) {
   return make_float2(M, a.y * ex2(a.x - M) + b.y * ex2(b.x - M));
 }
 
+// The d-th dynamic head, scanning on from a cursor (cd, clh) = (index, head)
+// of the last one found; -1 when there is none.
+__device__ __forceinline__ int dyn_head(const uint8_t* __restrict__ role, int LH, int d, int& cd,
+                                        int& clh) {
+  if (d < cd) {
+    cd = -1;
+    clh = -1;
+  }
+  while (cd < d) {
+    ++clh;
+    while (clh < LH && !role[clh]) ++clh;
+    if (clh >= LH) return -1;
+    ++cd;
+  }
+  return clh;
+}
+
+// Walks the units in order: dynamic head dh, query tile qt, block b of that
+// (head, tile) = block blk of frame f, or block b - F*nbf of the chunk.  One
+// division at the start, counters after.
+struct ScoreUnit {
+  int dh, qt, b, f, blk;
+  int row0;    // first key row of the block in its tensor
+  int nk;      // valid keys of the block (1..128)
+  bool chunk;  // the block is one of the chunk's own keys
+
+  __device__ __forceinline__ void at(const ScoreArgs& a, int64_t u) {
+    const int NB = a.F * a.nbf + a.nbc;
+    dh = int(u / (int64_t(a.n_qt) * NB));
+    const int rem = int(u - int64_t(dh) * a.n_qt * NB);
+    qt = rem / NB;
+    b = rem - qt * NB;
+    f = b / a.nbf;
+    blk = b - f * a.nbf;
+    derive(a);
+  }
+  __device__ __forceinline__ void next(const ScoreArgs& a) {
+    ++b;
+    if (++blk == a.nbf) {
+      blk = 0;
+      ++f;
+    }
+    if (b == a.F * a.nbf + a.nbc) {
+      b = f = blk = 0;
+      if (++qt == a.n_qt) {
+        qt = 0;
+        ++dh;
+      }
+    }
+    derive(a);
+  }
+  __device__ __forceinline__ void derive(const ScoreArgs& a) {
+    chunk = f >= a.F;
+    if (!chunk) {
+      row0 = f * a.T + blk * 128;
+      nk = min(128, a.T - blk * 128);
+    } else {
+      row0 = (b - a.F * a.nbf) * 128;
+      nk = min(128, a.Lq - row0);
+    }
+  }
+};
+
 __global__ void __launch_bounds__(kScoreThreads, 2)
 score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_kc, const ScoreArgs a) {
-  const int qt = blockIdx.x, g = blockIdx.y, lh = blockIdx.z;
-  if (!a.head_role[lh]) return;  // static head: nothing to score (uniform per CTA)
-  // Key range of this CTA: a history sub-segment, or (last entry) the chunk's
-  // own keys when they join the normaliser.
-  const bool chunk = g >= a.G;
-  const CUtensorMap* tmk = chunk ? &tm_kc : &tm_k;
-  int row0, nkeys;
-  if (chunk) {
-    row0 = 0;
-    nkeys = a.Lq;
-  } else {
-    // sub-segment `sub` of frame f: its blocks [bs, be) of the frame's nbf,
-    // bs = ceil(sub * nbf / split) (equal frames are cut at the same blocks)
-    const int f = g / kScoreSplit, sub = g - f * kScoreSplit;
-    const int nbf = (a.T + 127) / 128;
-    const int bs = (sub * nbf + kScoreSplit - 1) / kScoreSplit;
-    const int be = ((sub + 1) * nbf + kScoreSplit - 1) / kScoreSplit;
-    row0 = f * a.T + bs * 128;
-    nkeys = (be * 128 < a.T ? be * 128 : a.T) - bs * 128;
-  }
-  const int b0 = 0, b1 = nkeys > 0 ? (nkeys + 127) / 128 : 0;
-  float2* out = a.part_ml + (int64_t(lh) * a.E + g) * a.n_s;
-  if (b0 >= b1) {  // empty sub-segment (a frame of one block): neutral statistics
-    const int64_t i = int64_t(qt) * 128 + threadIdx.x;
-    if (threadIdx.x < 128 && i < a.n_s) out[i] = make_float2(-INFINITY, 0.f);
-    return;
-  }
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = align1024(smem_raw);
   ScoreBars* bars = reinterpret_cast<ScoreBars*>(sm + kSOffBar);
@@ -115,17 +157,27 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < kScoreStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->s_full[b], 1);
-      mbar_init(&bars->s_free[b], kScoreStatThreads);
+      mbar_init(&bars->s_free[b], 2 * kScoreHalfThreads);
+      mbar_init(&bars->x_full[b], kScoreHalfThreads);
+      mbar_init(&bars->x_read[b], kScoreHalfThreads);
     }
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
+    bars->n_dyn = 0;
     fence_mbar_init();
+  }
+  __syncthreads();
+  {  // dynamic heads: the units cover only them
+    int c = 0;
+    for (int i = threadIdx.x; i < a.LH; i += blockDim.x) c += a.head_role[i] != 0;
+    if (c) atomicAdd(&bars->n_dyn, c);
   }
   if (warp == kScoreMmaWarp) {
     tmem_alloc(&bars->tmem_base, 256);
@@ -134,34 +186,63 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-  const int row = (warp & 3) * 32 + lane, half = warp >> 2;
-  float m = -INFINITY, l = 0.f;
+  const int64_t NB = int64_t(a.F) * a.nbf + a.nbc;
+  const int64_t U = int64_t(bars->n_dyn) * a.n_qt * NB;
+  const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
 
   if (warp == kScoreProducerWarp) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       prefetch_tmap(&tm_qs);
-      prefetch_tmap(tmk);
-      mbar_expect_tx(&bars->q_full, kTileBytes);
-      tma_load_tile(sm + kSOffQ, &tm_qs, &bars->q_full, qt * 128, lh);
-      uint32_t issued = 0;
-      for (int b = b0; b < b1; ++b, ++issued) {
-        const uint32_t s = issued % kScoreStages, u = issued / kScoreStages;
-        if (!mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort)) break;
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_kc);
+      int cd = -1, clh = -1, prev = -1;
+      uint32_t qn = 0, kn = 0;
+      bool ok = true;
+      ScoreUnit t;
+      if (u0 < u1) t.at(a, u0);
+      for (int64_t u = u0; ok && u < u1; ++u, t.next(a)) {
+        const int lh = dyn_head(a.head_role, a.LH, t.dh, cd, clh);
+        if (lh < 0) break;
+        const int key = t.dh * a.n_qt + t.qt;
+        if (key != prev) {  // a new query tile once the MMAs on the last one are done
+          if (qn > 0 && !(ok = mbar_wait(&bars->q_empty, (qn - 1) & 1, abort))) break;
+          mbar_expect_tx(&bars->q_full, kTileBytes);
+          tma_load_tile(sm + kSOffQ, &tm_qs, &bars->q_full, t.qt * 128, lh);
+          ++qn;
+          prev = key;
+        }
+        const uint32_t s = kn % kScoreStages, use = kn / kScoreStages;
+        if (!(ok = mbar_wait(&bars->k_empty[s], (use & 1) ^ 1, abort))) break;
         mbar_expect_tx(&bars->k_full[s], kTileBytes);
-        tma_load_tile(sm + kSOffK + s * kTileBytes, tmk, &bars->k_full[s], row0 + b * 128, lh);
+        tma_load_tile(sm + kSOffK + s * kTileBytes, t.chunk ? &tm_kc : &tm_k, &bars->k_full[s],
+                      t.row0, lh);
+        ++kn;
       }
-      for (uint32_t i = issued > kScoreStages ? issued - kScoreStages : 0; i < issued; ++i)
+      for (uint32_t i = kn > kScoreStages ? kn - kScoreStages : 0; i < kn; ++i)
         drain_wait_s(&bars->k_full[i % kScoreStages], (i / kScoreStages) & 1);
-      drain_wait_s(&bars->q_full, 0);
+      if (qn > 0) drain_wait_s(&bars->q_full, (qn - 1) & 1);
     }
   } else if (warp == kScoreMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      bool ok = mbar_wait(&bars->q_full, 0, abort);
       const uint32_t qbase = smem_u32(sm + kSOffQ);
-      for (uint32_t it = 0; ok && it < uint32_t(b1 - b0); ++it) {
-        const uint32_t s = it % kScoreStages, u = it / kScoreStages;
+      int prev = -1;
+      uint32_t qn = 0, it = 0;
+      bool ok = true;
+      ScoreUnit t;
+      if (u0 < u1) t.at(a, u0);
+      for (int64_t u = u0; ok && u < u1; ++u, ++it, t.next(a)) {
+        const int key = t.dh * a.n_qt + t.qt;
+        if (key != prev) {
+          if (qn > 0) mma_commit(&bars->q_empty);  // arrives when the last tile's MMAs are done
+          if (!(ok = mbar_wait(&bars->q_full, qn & 1, abort))) break;
+          ++qn;
+          prev = key;
+        }
+        const uint32_t s = it % kScoreStages, use = it / kScoreStages;
         const uint32_t sb = it & 1, su = it >> 1;
-        if (!(ok = mbar_wait(&bars->k_full[s], u & 1, abort))) break;
+        if (!(ok = mbar_wait(&bars->k_full[s], use & 1, abort))) break;
         if (!(ok = mbar_wait(&bars->s_free[sb], (su & 1) ^ 1, abort))) break;
         tc_fence_after();
         const uint32_t kbase = smem_u32(sm + kSOffK + s * kTileBytes);
@@ -176,12 +257,19 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
       drain_wait_s(&bars->mma_done, 0);
     }
   } else {
+    // ------------------------------------------------------------ statistics warps
+    const int row = (warp & 3) * 32 + lane, half = warp >> 2;
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const float2 sl2x2 = make_float2(a.sl2, a.sl2);
+    int cd = -1, clh = -1;
+    uint32_t it = 0;
     bool ok = true;
-    for (uint32_t it = 0; ok && it < uint32_t(b1 - b0); ++it) {
+    ScoreUnit t;
+    if (u0 < u1) t.at(a, u0);
+    for (int64_t u = u0; ok && u < u1; ++u, ++it, t.next(a)) {
+      const int lh = dyn_head(a.head_role, a.LH, t.dh, cd, clh);
       const uint32_t sb = it & 1, su = it >> 1;
-      const int cols_left = nkeys - int(it) * 128 - 64 * half;
+      const int cols_left = t.nk - 64 * half;
       const int nv = cols_left < 0 ? 0 : (cols_left < 64 ? cols_left : 64);
       if (!(ok = warp_wait_s(&bars->s_full[sb], su & 1, abort))) break;
       tc_fence_after();
@@ -191,7 +279,7 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
       tmem_ld_wait();
       tc_fence_before();
       mbar_arrive(&bars->s_free[sb]);
-      if (nv < 64) {  // columns past the frame's last token never count
+      if (nv < 64) {  // columns past the block's last key never count
 #pragma unroll
         for (int i = 0; i < 64; ++i)
           if (i >= nv) r[i] = 0xff800000u;  // -inf
@@ -206,8 +294,8 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
           mx[k] = fmax3(mx[k], __uint_as_float(r[i + k]), __uint_as_float(r[i + k + 8]));
       const float bmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
                                fmaxf(mx[6], mx[7]));
-      const float m_new = fmaxf(m, bmax * a.sl2);  // scale > 0
-      const float mref = m_new == -INFINITY ? 0.f : m_new;
+      const float m = bmax * a.sl2;  // scale > 0; -inf for an empty half
+      const float mref = m == -INFINITY ? 0.f : m;
       const float2 negm2 = make_float2(-mref, -mref);
       float2 acc[4];
 #pragma unroll
@@ -219,22 +307,29 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
         acc[i & 3] = fadd2(acc[i & 3], make_float2(ex2(e.x), ex2(e.y)));
       }
       const float2 s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-      l = (m == -INFINITY ? 0.f : l * ex2(m - mref)) + (s2.x + s2.y);
-      m = m_new;
+      const float2 mine = make_float2(m, m == -INFINITY ? 0.f : s2.x + s2.y);
+      // merge the two column halves of the row; half 0 writes the entry
+      if (half) {
+        if (!(ok = warp_wait_s(&bars->x_read[sb], (su & 1) ^ 1, abort))) break;
+        bars->xml[sb][row] = mine;
+        mbar_arrive(&bars->x_full[sb]);
+      } else {
+        if (!(ok = warp_wait_s(&bars->x_full[sb], su & 1, abort))) break;
+        const float2 other = bars->xml[sb][row];
+        mbar_arrive(&bars->x_read[sb]);
+        const int64_t i = int64_t(t.qt) * 128 + row;
+        if (lh >= 0 && i < a.n_s)
+          a.part_ml[(int64_t(lh) * a.n_s + i) * a.E + t.b] = merge_ml(mine, other);
+      }
     }
-    bars->xml[half][row] = make_float2(m, l);
   }
 
   __syncthreads();
-  if (warp < 4 && !*abort) {
-    const int64_t i = int64_t(qt) * 128 + row;
-    if (i < a.n_s) out[i] = merge_ml(bars->xml[0][row], bars->xml[1][row]);
-  }
   if (warp == kScoreMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
-  if (threadIdx.x == 0 && *abort) report(a.status, FKV_ERR_TIMEOUT, lh);
+  if (threadIdx.x == 0 && *abort) report(a.status, FKV_ERR_TIMEOUT, blockIdx.x);
 }
 
 }  // namespace sm100
@@ -253,12 +348,16 @@ cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const voi
   } else {
     tkc = tk;  // never read
   }
+  const ScoreLayout sl = score_layout(d);
   ScoreArgs a;
+  a.LH = d.LH;
   a.T = d.T;
-  a.G = d.F * kScoreSplit;
-  a.E = a.G + 1;
+  a.F = d.F;
+  a.nbf = sl.split;
+  a.nbc = sl.chunk;
+  a.E = sl.E;
+  a.n_qt = int((d.n_s + 127) / 128);
   a.Lq = int(d.Lq);
-  a.with_chunk = d.score_with_chunk ? 1 : 0;
   a.n_s = d.n_s;
   a.sl2 = d.scale * 1.4426950408889634f;
   a.head_role = head_role;
@@ -267,8 +366,12 @@ cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const voi
   cudaError_t e = cudaFuncSetAttribute(score_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(kScoreSmem));
   if (e != cudaSuccess) return e;
-  dim3 grid(unsigned((d.n_s + 127) / 128), unsigned(a.G + a.with_chunk), unsigned(d.LH));
-  score_sm100_kernel<<<grid, kScoreThreads, kScoreSmem, s>>>(tqs, tk, tkc, a);
+  // Persistent: two CTAs per SM, fewer when there are fewer units than that.
+  const int64_t units_max = int64_t(d.LH) * a.n_qt * (int64_t(d.F) * a.nbf + a.nbc);
+  int64_t grid = int64_t(num_sms()) * 2;
+  if (units_max < grid) grid = units_max;
+  if (grid < 1) return cudaSuccess;
+  score_sm100_kernel<<<unsigned(grid), kScoreThreads, kScoreSmem, s>>>(tqs, tk, tkc, a);
   return cudaGetLastError();
 }
 

@@ -103,44 +103,47 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
     l = l * exp2f(m - mn) + ps;
     m = mn;
   }
-  if (c8 == 0 && r < nq) part_ml[(int64_t(lh) * (F + 1) + f) * n_s + row0 + r] = make_float2(m, l);
+  if (c8 == 0 && r < nq) part_ml[(int64_t(lh) * n_s + row0 + r) * (F + 1) + f] = make_float2(m, l);
 }
 
-// Frame masses from the partial statistics of G = F*split sub-segments per
-// head (split consecutive sub-segments per frame, then the chunk's own entry
-// when it joins the normaliser):
+// Frame masses from the partial statistics (layout of score_layout: F*split
+// frame entries per head, split consecutive pieces per frame, then `chunk`
+// entries of the chunk's own keys when they join the normaliser; G = F*split +
+// chunk entries in the row normaliser):
 //   row merge   M_i = max_g m_{g,i},  L_i = sum_g l_{g,i} 2^(m_{g,i} - M_i)
 //               (stored as (M_i, 1/L_i) in row_ml),
 //   frame mass  mass_f = sum_i c_{f,i},  c_{f,i} = sum_{g in f} l_{g,i} 2^(m_{g,i} - M_i) / L_i.
 // Two kernels, every sum in a fixed order (deterministic, equal frames give
 // bit-equal masses):
-//   score_rows_kernel    one warp per (head, row): lanes stride the entries,
-//                        a fixed shuffle tree; c_{f,i} is written back over
-//                        the m of the frame's first sub-segment of the same
-//                        row (each warp touches only its own row);
-//   score_frames_kernel  one warp per (head, frame): lanes stride the rows,
-//                        a fixed shuffle tree.
+//   score_rows_kernel    one warp per (head, row): lanes stride the row's
+//                        entries (contiguous), a fixed shuffle tree; c_{f,i}
+//                        is written back over the m of the frame's first
+//                        entry of the same row (each warp touches only its
+//                        own row);
+//   score_frames_kernel  one CTA per (head, frame): threads stride the rows,
+//                        a fixed shuffle tree and a fixed warp order.
 constexpr int kRowWarps = 8;
-constexpr int kFinThreads = 1024;
 
 __global__ void __launch_bounds__(kRowWarps * 32)
-score_rows_kernel(int F, int split, int with_chunk, int64_t n_s,
+score_rows_kernel(int F, int split, int chunk, int E, int64_t n_s,
                   const uint8_t* __restrict__ head_role, float2* __restrict__ part_ml,
                   float2* __restrict__ row_ml) {
   const int lh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t i = int64_t(blockIdx.x) * kRowWarps + warp;
   if (!head_role[lh] || i >= n_s) return;  // warp-uniform
-  const int G = F * split + with_chunk;
-  const int E = F * split + 1;
-  float2* p = part_ml + int64_t(lh) * E * n_s + i;
+  const int G = F * split + chunk;  // entries of the row normaliser
+  float2* p = part_ml + (int64_t(lh) * n_s + i) * E;  // the row's E entries, contiguous
+  // the entry loops are unrolled so that several loads are in flight per lane
   float M = -INFINITY;
-  for (int g = lane; g < G; g += 32) M = fmaxf(M, p[int64_t(g) * n_s].x);
+#pragma unroll 4
+  for (int g = lane; g < G; g += 32) M = fmaxf(M, p[g].x);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float Ls = 0.f;
+#pragma unroll 4
   for (int g = lane; g < G; g += 32) {
-    const float2 ml = p[int64_t(g) * n_s];
+    const float2 ml = p[g];
     if (ml.y != 0.f) Ls += ml.y * exp2f(ml.x - M);
   }
 #pragma unroll
@@ -155,8 +158,9 @@ score_rows_kernel(int F, int split, int with_chunk, int64_t n_s,
       c[u] = 0.f;
       if (f < F) {
         float t = 0.f;
+#pragma unroll 4
         for (int s2 = 0; s2 < split; ++s2) {
-          const float2 ml = p[int64_t(f * split + s2) * n_s];
+          const float2 ml = p[f * split + s2];
           if (ml.y != 0.f) t += ml.y * exp2f(ml.x - M);
         }
         c[u] = t * inv;
@@ -166,31 +170,37 @@ score_rows_kernel(int F, int split, int with_chunk, int64_t n_s,
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int f = f0 + lane + 32 * u;
-      if (f < F) p[int64_t(f * split) * n_s].x = c[u];
+      if (f < F) p[f * split].x = c[u];
     }
   }
 }
 
-__global__ void __launch_bounds__(kFinThreads)
-score_frames_kernel(int F, int split, int64_t n_s, const uint8_t* __restrict__ head_role,
+// One CTA per (head, frame): thread t sums rows t, t + 256, ... in order, then
+// a fixed shuffle tree per warp and the warp sums in warp order.
+constexpr int kFrameThreads = 256;
+
+__global__ void __launch_bounds__(kFrameThreads)
+score_frames_kernel(int F, int split, int E, int64_t n_s, const uint8_t* __restrict__ head_role,
                     const float2* __restrict__ part_ml, float* __restrict__ seg_score) {
-  const int lh = blockIdx.x;
-  const int E = F * split + 1;
-  float* out = seg_score + int64_t(lh) * F;
+  __shared__ float wsum[kFrameThreads / 32];
+  const int f = blockIdx.x, lh = blockIdx.y;
+  float* out = seg_score + int64_t(lh) * F + f;
   if (!head_role[lh]) {
-    for (int f = threadIdx.x; f < F; f += blockDim.x) out[f] = 0.f;
+    if (threadIdx.x == 0) *out = 0.f;
     return;
   }
-  const float2* p = part_ml + int64_t(lh) * E * n_s;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int f = warp; f < F; f += blockDim.x >> 5) {
-    const float2* cf = p + int64_t(f * split) * n_s;
-    float acc = 0.f;
+  const float2* cf = part_ml + int64_t(lh) * n_s * E + f * split;
+  float acc = 0.f;
 #pragma unroll 4
-    for (int64_t i = lane; i < n_s; i += 32) acc += cf[i].x;
+  for (int64_t i = threadIdx.x; i < n_s; i += kFrameThreads) acc += cf[i * E].x;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) out[f] = acc;
+  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+    for (int w = 0; w < kFrameThreads / 32; ++w) t += wsum[w];
+    *out = t;
   }
 }
 
@@ -213,18 +223,19 @@ cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void
   return cudaGetLastError();
 }
 
-cudaError_t launch_score_frame_finalize(const Dims& d, int split, const uint8_t* head_role,
-                                        float2* part_ml, float2* row_ml, float* seg_score,
-                                        cudaStream_t s) {
+cudaError_t launch_score_frame_finalize(const Dims& d, const ScoreLayout& sl,
+                                        const uint8_t* head_role, float2* part_ml,
+                                        float2* row_ml, float* seg_score, cudaStream_t s) {
   if (d.n_s > 0) {
     dim3 grid(unsigned((d.n_s + kRowWarps - 1) / kRowWarps), unsigned(d.LH));
-    score_rows_kernel<<<grid, kRowWarps * 32, 0, s>>>(d.F, split, d.score_with_chunk ? 1 : 0,
-                                                      d.n_s, head_role, part_ml, row_ml);
+    score_rows_kernel<<<grid, kRowWarps * 32, 0, s>>>(d.F, sl.split, sl.chunk, sl.E, d.n_s,
+                                                      head_role, part_ml, row_ml);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  score_frames_kernel<<<d.LH, kFinThreads, 0, s>>>(d.F, split, d.n_s, head_role, part_ml,
-                                                   seg_score);
+  if (d.F < 1) return cudaSuccess;
+  score_frames_kernel<<<dim3(unsigned(d.F), unsigned(d.LH)), kFrameThreads, 0, s>>>(
+      d.F, sl.split, sl.E, d.n_s, head_role, part_ml, seg_score);
   return cudaGetLastError();
 }
 

@@ -143,9 +143,16 @@ def test_param_validation(lib):
 def test_derived_sizes(lib):
     s = fkv.sizes(_p())
     assert s["nseg"] == 6 and s["max_kept"] == 6 and s["max_comp_rows"] == 192
-    # status block + (max, sum) per frame and scoring row + (max, sum) per row
-    # 2 sub-segments per frame + the chunk entry, then per-row merges
-    assert s["ws_bytes"] == 256 + 4 * (6 * 2 + 1) * 32 * 8 + 4 * 32 * 8
+    # status block + (max, sum) per 128-key block of each frame and scoring
+    # row (T = 32: one block per frame, no chunk entries), then per-row merges
+    assert s["ws_bytes"] == 256 + 4 * 6 * 32 * 8 + 4 * 32 * 8
+    # T = 300 (3 blocks per frame) with the chunk's 3 blocks in the normaliser
+    a256 = lambda n: (n + 255) // 256 * 256  # noqa: E731  (each region 256-byte aligned)
+    c = fkv.sizes(_p(T=300, score_with_chunk=True))
+    assert c["ws_bytes"] == 256 + a256(4 * (6 * 3 + 3) * 300 * 8) + a256(4 * 300 * 8)
+    # fp32 (CUDA-core) scoring: one entry per frame + one chunk slot
+    f = fkv.sizes(_p(dtype="fp32", D=64))
+    assert f["ws_bytes"] == 256 + 4 * (6 + 1) * 32 * 8 + 4 * 32 * 8
     t = fkv.sizes(_p(granularity="token", sink_tokens=40, recent_tokens=40, n_score_q=8))
     assert t["nseg"] == 192 - 80 and t["max_kept"] == 192 and t["max_comp_rows"] == 192
 

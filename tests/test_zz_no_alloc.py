@@ -64,7 +64,7 @@ def test_noalloc_matches_workspace_scoring_twice(cuda_device, case):
 
 
 def test_noalloc_rejects_scratch_above_its_maximum(cuda_device):
-    w = wl.get("480p_30layer")  # 30 layers of partial statistics: about 15 MB
+    w = wl.get("480p_30layer")  # 30 layers of per-block partial statistics: about 200 MB
     p = fkv.params_for(w)
     assert fkv.sizes(p)["ws_bytes"] > 4 << 20
     sentinel = torch.full((w.L, w.H, w.F), 7.0, device="cuda")

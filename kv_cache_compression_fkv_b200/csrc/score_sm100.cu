@@ -13,7 +13,7 @@
 // in a fixed order.  Equal frames are therefore reduced in exactly the same
 // order (bit-equal masses) however the units are spread over CTAs.
 //
-// The grid is persistent (two CTAs per SM): the dynamic heads are counted on
+// The grid is persistent (two CTAs per SM by default): the dynamic heads are counted on
 // the device and CTA c takes units [c*U/G, (c+1)*U/G) of the U units, ordered
 // (dynamic head, query tile, block), so the work is balanced to one block and
 // the K pipeline runs on across units.  Warp roles (320 threads): warps 0-7
@@ -29,7 +29,15 @@
 namespace fkv {
 namespace sm100 {
 
-constexpr int kScoreStages = 2;
+// K ring depth and CTAs per SM (shared memory: 32 KB per stage + 32 KB of Q).
+#ifndef FKV_SCORE_STAGES
+#define FKV_SCORE_STAGES 2
+#endif
+#ifndef FKV_SCORE_CTAS_PER_SM
+#define FKV_SCORE_CTAS_PER_SM 2
+#endif
+constexpr int kScoreStages = FKV_SCORE_STAGES;
+constexpr int kScoreCtasPerSm = FKV_SCORE_CTAS_PER_SM;
 constexpr int kScoreThreads = 320;
 constexpr int kScoreHalfThreads = 128;  // one column half of the statistics warps
 constexpr int kScoreProducerWarp = 8;
@@ -145,7 +153,7 @@ struct ScoreUnit {
   }
 };
 
-__global__ void __launch_bounds__(kScoreThreads, 2)
+__global__ void __launch_bounds__(kScoreThreads, kScoreCtasPerSm)
 score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_kc, const ScoreArgs a) {
@@ -368,7 +376,7 @@ cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const voi
   if (e != cudaSuccess) return e;
   // Persistent: two CTAs per SM, fewer when there are fewer units than that.
   const int64_t units_max = int64_t(d.LH) * a.n_qt * (int64_t(d.F) * a.nbf + a.nbc);
-  int64_t grid = int64_t(num_sms()) * 2;
+  int64_t grid = int64_t(num_sms()) * kScoreCtasPerSm;
   if (units_max < grid) grid = units_max;
   if (grid < 1) return cudaSuccess;
   score_sm100_kernel<<<unsigned(grid), kScoreThreads, kScoreSmem, s>>>(tqs, tk, tkc, a);

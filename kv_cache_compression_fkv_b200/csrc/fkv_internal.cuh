@@ -60,8 +60,8 @@ inline ScoreLayout score_layout(const Dims& d) {
 // Workspace layout (byte offsets from the workspace base, 256-B aligned).
 struct WsLayout {
   size_t status;     // int32[2]: first device error, detail
-  size_t part_ml;    // frame mode: float2 [LH][F*kScoreSplit + 1][n_s] per-sub-segment
-                     // (max, sum); the last entry is the chunk's own keys
+  size_t part_ml;    // frame mode: float2 [LH][n_s][E] (max, sum) per entry, the
+                     // layout of score_layout()
   size_t row_ml;     // frame mode: float2 [LH][n_s] per-row (max, sum)
   size_t qbar;       // token mode: float [LH][D] summed scoring queries
   size_t total;

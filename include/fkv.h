@@ -54,8 +54,8 @@ extern "C" {
 #endif
 
 /* 3: adds fkv_fp8_cache_t and the three *_fp8 entry points;
- * 4: adds fkv_select_heuristic. */
-#define FKV_ABI_VERSION 4
+ * 4: adds fkv_select_heuristic; 5: adds fkv_step_fp8. */
+#define FKV_ABI_VERSION 5
 
 typedef enum fkv_status {
   FKV_OK = 0,
@@ -389,6 +389,16 @@ int32_t fkv_quantize_chunk_fp8(const fkv_params_t* p, const void* q_cur, const v
  * attention over the dequantised cache by that rounding. */
 int32_t fkv_attend_compressed_fp8(const fkv_params_t* p, const fkv_fp8_cache_t* c,
                                   const int32_t* kept_cnt, void* out, void* ws, void* stream);
+
+/* Steps 1-5 with the e4m3 cache in one call: score and select as fkv_step,
+ * then fkv_compact_gather_fp8, fkv_quantize_chunk_fp8 and
+ * fkv_attend_compressed_fp8, all enqueued on `stream` in that order.  io as
+ * for fkv_step (frame mode), except that io->k_comp / io->v_comp are not used
+ * (may be NULL); c holds every e4m3 operand.  Same support limits as
+ * fkv_attend_compressed_fp8; every host-side check runs before the first
+ * launch. */
+int32_t fkv_step_fp8(const fkv_params_t* p, const fkv_step_io_t* io, const fkv_fp8_cache_t* c,
+                     void* ws, void* stream);
 
 #ifdef __cplusplus
 }

@@ -414,6 +414,19 @@ def attend_compressed_fp8(p: Params, cache, kept_cnt, out, ws, stream=None):
     _check(st, "fkv_attend_compressed_fp8")
 
 
+def step_fp8(p: Params, inputs: Dict[str, torch.Tensor], outputs: Dict[str, torch.Tensor],
+             cache: Dict[str, torch.Tensor], stream=None, io: Optional[StepIO] = None):
+    """The whole chunk step with the e4m3 cache (fkv_step_fp8): ``inputs`` and
+    ``outputs`` as for :func:`step` (the bf16 k_comp / v_comp are not used),
+    ``cache`` from :func:`allocate_fp8`."""
+    if io is None:
+        io = make_step_io(p, inputs, outputs)
+    fp = make_fp8_cache(p, cache)
+    st = _lib.load().fkv_step_fp8(ctypes.byref(p), ctypes.byref(io), ctypes.byref(fp),
+                                  outputs["ws"].data_ptr(), _stream(stream))
+    _check(st, "fkv_step_fp8")
+
+
 def read_status(ws: torch.Tensor, stream=None):
     """(first device-side status since init, (layer*H + head) it was seen on or -1).
     Synchronises the stream."""

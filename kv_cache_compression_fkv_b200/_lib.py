@@ -93,6 +93,8 @@ SIGNATURES = {
                                        ctypes.POINTER(Fp8Cache), c_vp, c_vp]),
     "fkv_attend_compressed_fp8": (c_i32, [ctypes.POINTER(Params), ctypes.POINTER(Fp8Cache), c_vp,
                                           c_vp, c_vp, c_vp]),
+    "fkv_step_fp8": (c_i32, [ctypes.POINTER(Params), ctypes.POINTER(StepIO), ctypes.POINTER(Fp8Cache),
+                             c_vp, c_vp]),
 }
 
 _lib = None

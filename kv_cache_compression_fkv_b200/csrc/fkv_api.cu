@@ -487,6 +487,27 @@ int32_t fkv_quantize_chunk_fp8(const fkv_params_t* p, const void* q_cur, const v
   return cuda_status(launch_quant_rows(d, q_cur, c->q_cur, c->q_scale, s));
 }
 
+// Host-side checks of the e4m3 operands that the given steps use.
+static int32_t check_fp8_cache(const Dims& d, const fkv_fp8_cache_t* c, bool comp, bool cur) {
+  if (!c) return FKV_ERR_INVALID_ARG;
+  if (comp) {
+    if (((!c->k_comp || !c->v_comp) && d.comp_rows > 0) ||
+        ((!c->k_comp_scale || !c->v_comp_scale) && d.F > 0))
+      return FKV_ERR_INVALID_ARG;
+    if (!aligned16(c->k_comp) || !aligned16(c->v_comp) || !aligned4(c->k_comp_scale) ||
+        !aligned4(c->v_comp_scale))
+      return FKV_ERR_INVALID_ARG;
+  }
+  if (cur) {
+    if (!c->q_cur || !c->q_scale || !c->k_cur || !c->v_cur || !c->k_cur_scale || !c->v_cur_scale)
+      return FKV_ERR_INVALID_ARG;
+    if (!aligned16(c->q_cur) || !aligned16(c->k_cur) || !aligned16(c->v_cur) ||
+        !aligned4(c->q_scale) || !aligned4(c->k_cur_scale) || !aligned4(c->v_cur_scale))
+      return FKV_ERR_INVALID_ARG;
+  }
+  return FKV_OK;
+}
+
 int32_t fkv_attend_compressed_fp8(const fkv_params_t* p, const fkv_fp8_cache_t* c,
                                   const int32_t* kept_cnt, void* out, void* ws, void* stream) {
   Dims d;
@@ -506,6 +527,44 @@ int32_t fkv_attend_compressed_fp8(const fkv_params_t* p, const fkv_fp8_cache_t* 
   if (d.LH == 0 || d.Lq == 0) return FKV_OK;
   return cuda_status(launch_attend_fp8_sm100(d, *c, kept_cnt, out, status_ptr(ws),
                                              static_cast<cudaStream_t>(stream)));
+}
+
+int32_t fkv_step_fp8(const fkv_params_t* p, const fkv_step_io_t* io, const fkv_fp8_cache_t* c,
+                     void* ws, void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (!fp8_supported(d) || d.T < 128) return FKV_ERR_UNSUPPORTED;
+  if (!io) return FKV_ERR_INVALID_ARG;
+  // every check before the first launch
+  if (!io->q_cur || !io->k_cur || !io->v_cur || ((!io->k_hist || !io->v_hist) && d.N > 0) ||
+      !io->k_per_head || (!io->seg_score && d.nseg > 0) || (!io->kept_idx && d.max_kept > 0) ||
+      !io->kept_cnt || !io->out || !io->head_role || (!io->static_mask && d.F > 0))
+    return FKV_ERR_INVALID_ARG;
+  const void* ptrs[] = {io->q_cur, io->k_cur, io->v_cur, io->k_hist, io->v_hist, io->out};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FKV_ERR_INVALID_ARG;
+  if ((st = check_fp8_cache(d, c, true, true)) != FKV_OK) return st;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = do_score(d, io->q_cur, io->q_score, io->k_hist, io->k_cur, io->head_role,
+                     io->seg_score, ws, s)))
+    return st;
+  if ((st = do_select(d, io->seg_score, io->head_role, io->static_mask, io->k_per_head,
+                      io->kept_idx, io->kept_cnt, ws, s)))
+    return st;
+  if (d.F > 0 &&
+      (st = cuda_status(launch_quant_segments(d, int(d.max_kept), d.N, d.comp_rows, io->kept_idx,
+                                              io->kept_cnt, io->k_hist, io->v_hist, c->k_comp,
+                                              c->v_comp, c->k_comp_scale, c->v_comp_scale,
+                                              status_ptr(ws), s))))
+    return st;
+  if ((st = cuda_status(launch_quant_segments(d, d.Fc, d.Lq, d.Lq, nullptr, nullptr, io->k_cur,
+                                              io->v_cur, c->k_cur, c->v_cur, c->k_cur_scale,
+                                              c->v_cur_scale, status_ptr(ws), s))))
+    return st;
+  if ((st = cuda_status(launch_quant_rows(d, io->q_cur, c->q_cur, c->q_scale, s)))) return st;
+  return cuda_status(launch_attend_fp8_sm100(d, *c, io->kept_cnt, io->out, status_ptr(ws), s));
 }
 
 }  // extern "C"

@@ -97,7 +97,7 @@ def test_fp8_entry_points_validate_before_launch(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fkv_abi_version() == 4
+    assert lib.fkv_abi_version() == 5
     for code in range(8):
         assert lib.fkv_status_string(code).decode().startswith("FKV_")
     assert lib.fkv_status_string(99) == b"FKV_ERR_UNKNOWN"
@@ -190,3 +190,18 @@ def test_heuristic_selector_validates_before_launch(lib):
     tm = _fp8_params(static_token_mask=True)
     assert lib.fkv_select_heuristic(ctypes.byref(tm), _lib.FKV_POLICY_UNIFORM, 1, fake, None, fake,
                                     fake, fake, None) == _lib.FKV_ERR_UNSUPPORTED
+
+
+def test_step_fp8_validates_before_launch(lib):
+    p = _fp8_params()
+    io = _lib.StepIO()
+    c = _lib.Fp8Cache()
+    fake = ctypes.c_void_p(1 << 20)
+    assert lib.fkv_step_fp8(ctypes.byref(p), None, ctypes.byref(c), fake, None) == _lib.FKV_ERR_INVALID_ARG
+    for f in _lib.STEP_IO_FIELDS:
+        setattr(io, f, 1 << 20)
+    # the e4m3 operands are checked before anything is launched
+    assert lib.fkv_step_fp8(ctypes.byref(p), ctypes.byref(io), ctypes.byref(c), fake, None) == _lib.FKV_ERR_INVALID_ARG
+    assert lib.fkv_step_fp8(ctypes.byref(p), ctypes.byref(io), None, fake, None) == _lib.FKV_ERR_INVALID_ARG
+    small_t = _fp8_params(T=64, comp_rows=4 * 64)
+    assert lib.fkv_step_fp8(ctypes.byref(small_t), ctypes.byref(io), ctypes.byref(c), fake, None) == _lib.FKV_ERR_UNSUPPORTED

@@ -145,3 +145,33 @@ def test_attend_fp8_480p_sampled_rows(cuda_device):
         # fp8 against bf16 operands: the quantisation error, well below the signal
         g16 = out16[l, h, rows].cpu().double().numpy()
         assert np.abs(got - g16).mean() <= 0.05 * np.abs(g16).mean()
+
+
+def test_step_fp8_equals_the_separate_calls(cuda_device):
+    w = wl.scaled(wl.get("480p"), name="step_fp8", H=4, T=256, F=6, Fc=2, n_static=2,
+                  static_frames=(0, 2, 5), k_dynamic=3, score_stride=4, seed=31)
+    x = parity.upload(wl.generate(w))
+    p = fkv.params_for(w)
+    o = fkv.allocate(p)
+    c = fkv.allocate_fp8(p)
+    fkv.step_fp8(p, x, o, c)
+    assert fkv.read_status(o["ws"])[0] == 0
+    # the same steps one call at a time
+    r = fkv.allocate(p)
+    c2 = fkv.allocate_fp8(p)
+    fkv.score_segments(p, x["q_cur"], None, x["k_hist"], x["head_role"], r["seg_score"], r["ws"])
+    fkv.select_topk(p, r["seg_score"], x["head_role"], x["static_mask"], x["k_per_head"],
+                    r["kept_idx"], r["kept_cnt"], r["ws"])
+    fkv.compact_gather_fp8(p, x["k_hist"], x["v_hist"], r["kept_idx"], r["kept_cnt"], c2, r["ws"])
+    fkv.quantize_chunk_fp8(p, x["q_cur"], x["k_cur"], x["v_cur"], c2, r["ws"])
+    out2 = torch.empty_like(r["out"])
+    fkv.attend_compressed_fp8(p, c2, r["kept_cnt"], out2, r["ws"])
+    assert fkv.read_status(r["ws"])[0] == 0
+    assert torch.equal(o["kept_cnt"], r["kept_cnt"]) and torch.equal(o["seg_score"], r["seg_score"])
+    assert torch.equal(o["out"], out2)
+    for k in ("k_cur", "v_cur", "q_cur", "q_scale", "k_cur_scale", "v_cur_scale"):
+        assert torch.equal(c[k], c2[k]), k
+    cnt = o["kept_cnt"].cpu()
+    for h in range(w.H):
+        rows = int(cnt[0, h]) * w.T
+        assert torch.equal(c["k_comp"][0, h, :rows], c2["k_comp"][0, h, :rows])

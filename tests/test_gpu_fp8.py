@@ -175,3 +175,17 @@ def test_step_fp8_equals_the_separate_calls(cuda_device):
     for h in range(w.H):
         rows = int(cnt[0, h]) * w.T
         assert torch.equal(c["k_comp"][0, h, :rows], c2["k_comp"][0, h, :rows])
+
+
+def test_attend_fp8_1080p_sampled_rows(cuda_device):
+    w = wl.get("1080p")
+    x, p, d, o, c, kept_idx, kept_cnt = _setup(w, kept_seed=1080, n_keep=13)
+    out = torch.empty_like(o["out"])
+    fkv.attend_compressed_fp8(p, c, kept_cnt.cuda(), out, o["ws"])
+    assert fkv.read_status(o["ws"])[0] == 0
+    rows = wl.sample_rows(w.Fc * w.T, 24, seed=8)
+    for l, h in [(0, 2), (0, 9)]:
+        kept = kept_idx[l, h, :int(kept_cnt[l, h])].numpy()
+        ref, tol = _oracle_fp8_attention(x, w, l, h, kept, rows)
+        got = out[l, h, rows].cpu().double().numpy()
+        assert np.all(np.abs(got - ref) <= tol), (l, h)

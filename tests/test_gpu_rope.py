@@ -50,3 +50,27 @@ def test_compact_gather_rope(cuda_device, dtype, n_pairs):
                                   orc.compact(wl.as_float64(x["v_hist"][l, h]), kept, w.T))
             if n_pairs == 0:
                 assert np.array_equal(got_k, plain)
+
+
+def test_compact_gather_rope_480p(cuda_device):
+    w = wl.get("480p")
+    x = wl.generate(w)
+    p = fkv.params_for(w, comp_rows=w.F * w.T)
+    d = parity.upload(x)
+    o = fkv.allocate(p)
+    kept_idx, kept_cnt = wl.random_kept(w, seed=480, n_keep=13)
+    omega = torch.tensor(10000.0 ** (-np.arange(22) / 22), dtype=torch.float32)
+    kc = torch.full_like(o["k_comp"], float("nan"))
+    vc = torch.full_like(o["v_comp"], float("nan"))
+    fkv.compact_gather_rope(p, d["k_hist"], d["v_hist"], kept_idx.cuda(), kept_cnt.cuda(),
+                            omega.cuda(), kc, vc, o["ws"])
+    assert fkv.read_status(o["ws"])[0] == 0
+    for h in (0, 1, 5, 11):  # head 0 keeps nothing, head 1 every frame, the others 13
+        kept = kept_idx[0, h, :int(kept_cnt[0, h])].numpy()
+        rows = len(kept) * w.T
+        exp_k = orc.compact_repositioned(wl.as_float64(x["k_hist"][0, h]), kept, w.T, w.F,
+                                         omega.double().numpy())
+        got_k = kc[0, h, :rows].cpu().double().numpy()
+        assert np.all(np.abs(got_k - exp_k) <= 2.0 ** -8 * np.abs(exp_k) + 1e-6), h
+        assert np.array_equal(vc[0, h, :rows].cpu().double().numpy(),
+                              orc.compact(wl.as_float64(x["v_hist"][0, h]), kept, w.T))

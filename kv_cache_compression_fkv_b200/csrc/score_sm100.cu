@@ -56,6 +56,7 @@ struct ScoreBars {
   uint32_t tmem_base;
   int abort;
   int n_dyn;
+  int c_dh, c_lh;      // cursor: dynamic head c_dh is head c_lh (this CTA's first unit)
   float2 xml[2][128];  // [S buffer][row] (m, l) of the second column half
 };
 
@@ -197,6 +198,27 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
   const int64_t NB = int64_t(a.F) * a.nbf + a.nbc;
   const int64_t U = int64_t(bars->n_dyn) * a.n_qt * NB;
   const int64_t u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+  if (warp == 0) {  // the head of this CTA's first unit, 32 roles per ballot
+    int want = u0 < u1 ? int(u0 / (int64_t(a.n_qt) * NB)) : 0, found = -1;
+    const int dh0 = want;
+    for (int base = 0; base < a.LH && found < 0; base += 32) {
+      const int i = base + lane;
+      const bool dyn = i < a.LH && a.head_role[i] != 0;
+      const unsigned bits = __ballot_sync(0xffffffffu, dyn);
+      const int c = __popc(bits);
+      if (want < c) {
+        const int before = __popc(bits & ((1u << lane) - 1u));
+        found = base + __ffs(__ballot_sync(0xffffffffu, dyn && before == want)) - 1;
+      } else {
+        want -= c;
+      }
+    }
+    if (lane == 0) {
+      bars->c_dh = found >= 0 ? dh0 : -1;
+      bars->c_lh = found;
+    }
+  }
+  __syncthreads();
 
   if (warp == kScoreProducerWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -204,7 +226,7 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
       prefetch_tmap(&tm_qs);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_kc);
-      int cd = -1, clh = -1, prev = -1;
+      int cd = bars->c_dh, clh = bars->c_lh, prev = -1;
       uint32_t qn = 0, kn = 0;
       bool ok = true;
       ScoreUnit t;
@@ -269,7 +291,7 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
     const int row = (warp & 3) * 32 + lane, half = warp >> 2;
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const float2 sl2x2 = make_float2(a.sl2, a.sl2);
-    int cd = -1, clh = -1;
+    int cd = bars->c_dh, clh = bars->c_lh;
     uint32_t it = 0;
     bool ok = true;
     ScoreUnit t;

@@ -25,16 +25,24 @@
 //              rescaling: P stays <= 256, exact after the final merge).
 //              Exponentials run on the MUFU unit; FKV_POLY_EVERY = n sends
 //              one pair in n to the FMA-pipe polynomial exp2_poly2 instead
-//              (measured slower at 480P, where MUFU is ~45% busy: default 0).
+//              (measured slower at 480P: default 0).  The lead thread of
+//              each warpgroup releases the K stage of S_h(j) and the V stage
+//              of PV_h(j-1) once it sees S_h(j) complete.
 //   warp 8     TMA: lane 0 loads Q (once per unit) and the K blocks, lane 1
-//              the V blocks, into 3-stage rings in the order the MMAs use
-//              them: stream 0 block j, stream 1 block j, stream 0 block j+1...
+//              the V blocks, into rings (3 + 3 stages) in the order the MMAs
+//              use them: stream 0 block j, stream 1 block j, stream 0 block
+//              j+1...
 //   warp 9     MMA issuer (one thread) and TMEM owner.  Per step j it issues
 //              O_0 += P_0 V (block j-1), S_0 = Q K^T (block j), then the same
 //              for stream 1.  tcgen05 MMAs of one thread execute in issue
 //              order, so S_h of block j overwrites P_h only after the PV that
 //              reads it, and by the time S_h is complete the previous PV into
 //              O_h is complete too (the softmax may rescale O_h right away).
+//              The issuing thread is the pace-setter: it issues an M=128,
+//              N=128, K=16 MMA only slightly faster than the tensor core
+//              executes one and the hardware queue is short, so its work
+//              between MMA groups (each mbarrier test or commit costs it
+//              ~90 cycles) is kept to one wait and one commit per group.
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
 // Key blocks past the valid rows of a range are masked (logit -> -inf) and
@@ -49,7 +57,15 @@
 namespace fkv {
 namespace sm100 {
 
-constexpr int kKVStages = 3;
+#ifndef FKV_ATTN_K_STAGES
+#define FKV_ATTN_K_STAGES 3
+#endif
+#ifndef FKV_ATTN_V_STAGES
+#define FKV_ATTN_V_STAGES 3
+#endif
+// Ring depths of the K and V tiles (K + V = 6 tiles of 32 KB fit beside Q).
+constexpr int kKStages = FKV_ATTN_K_STAGES;
+constexpr int kVStages = FKV_ATTN_V_STAGES;
 constexpr int kAttnThreads = 384;        // 3 warpgroups
 // Register split (setmaxnreg): the kernel is launched with kLaunchRegs per
 // thread; the control warpgroup (TMA, MMA, two idle warps) gives registers
@@ -78,13 +94,13 @@ __host__ __device__ constexpr uint32_t col_o(int h) { return 256u + 128u * uint3
 
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kTileBytes;
-constexpr uint32_t kOffV = kOffK + kKVStages * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kKVStages * kTileBytes;
+constexpr uint32_t kOffV = kOffK + kKStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kVStages * kTileBytes;
 
 struct AttnBars {
   uint64_t q_full, q_empty;
-  uint64_t k_full[kKVStages], k_empty[kKVStages];
-  uint64_t v_full[kKVStages], v_empty[kKVStages];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], p_full[2];  // per stream
   uint64_t o_ready, o_free;       // per unit: both PV chains done / both O read
   uint64_t mma_done;
@@ -127,9 +143,11 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     mbar_init(&bars->q_empty, 1);
-    for (int s = 0; s < kKVStages; ++s) {
+    for (int s = 0; s < kKStages; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -174,7 +192,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int b = block_of(t, h, j);
             const bool inA = b < t.nbA;
             const int row = (inA ? b : b - t.nbA) * 128;
-            const uint32_t s = n % kKVStages, u = n / kKVStages;
+            const uint32_t s = n % kKStages, u = n / kKStages;
             if (!(ok = mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort))) break;
             mbar_expect_tx(&bars->k_full[s], kTileBytes);
             tma_load_tile(sm + kOffK + s * kTileBytes, inA ? &tm_kc : &tm_kn, &bars->k_full[s],
@@ -183,8 +201,8 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       }
-      for (uint32_t i = n > kKVStages ? n - kKVStages : 0; i < n; ++i)
-        drain_wait(&bars->k_full[i % kKVStages], (i / kKVStages) & 1);
+      for (uint32_t i = n > kKStages ? n - kKStages : 0; i < n; ++i)
+        drain_wait(&bars->k_full[i % kKStages], (i / kKStages) & 1);
       if (tc > 0) drain_wait(&bars->q_full, (tc - 1) & 1);
     } else if (lane == 1) {  // V
       prefetch_tmap(&tm_vc);
@@ -199,7 +217,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const int b = block_of(t, h, j);
             const bool inA = b < t.nbA;
             const int row = (inA ? b : b - t.nbA) * 128;
-            const uint32_t s = n % kKVStages, u = n / kKVStages;
+            const uint32_t s = n % kVStages, u = n / kVStages;
             if (!(ok = mbar_wait(&bars->v_empty[s], (u & 1) ^ 1, abort))) break;
             mbar_expect_tx(&bars->v_full[s], kTileBytes);
             tma_load_tile(sm + kOffV + s * kTileBytes, inA ? &tm_vc : &tm_vn, &bars->v_full[s],
@@ -208,63 +226,80 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
       }
-      for (uint32_t i = n > kKVStages ? n - kKVStages : 0; i < n; ++i)
-        drain_wait(&bars->v_full[i % kKVStages], (i / kKVStages) & 1);
+      for (uint32_t i = n > kVStages ? n - kVStages : 0; i < n; ++i)
+        drain_wait(&bars->v_full[i % kVStages], (i / kVStages) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // The tensor core queues only a few MMAs and one thread issues them barely
+    // faster than they execute, so whatever this thread does between two MMA
+    // groups leaves the tensor core idle.  It therefore only waits and
+    // issues: ring stages advance by cursors (K and V are consumed in load
+    // order), descriptors are precomputed, one commit per S group (the
+    // softmax releases the K and V stages), and a tcgen05 fence only where
+    // another thread wrote TMEM (P, and O after the epilogue).
     if (lane == 0) {
-      uint32_t n = 0, uc = 0;
+      uint32_t uc = 0, ks = 0, kph = 0, vs = 0, vph = 0;
       uint32_t p_use[2] = {0, 0};
       bool ok = true;
-      const uint32_t qbase = smem_u32(sm + kOffQ);
+      const uint64_t dq = kmajor_desc(smem_u32(sm + kOffQ), 0);
+      const uint64_t dk0 = kmajor_desc(smem_u32(sm + kOffK), 0);
+      const uint64_t dv0 = mnmajor_desc(smem_u32(sm + kOffV), 0);
+      constexpr uint32_t kStageDesc = kTileBytes >> 4;  // descriptor step between ring stages
       for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++uc) {
         const Unit t = decode(a, tile);
-        const uint32_t base = n;
         bool o_free_seen = false;
-        // O_h += P_h V for stream h's j-th block.
-        auto issue_pv = [&](int h, int j) -> bool {
+        // O_h += P_h V for the stream's next block (`first`: its first of the unit).
+        auto issue_pv = [&](int h, bool first) -> bool {
           if (!o_free_seen) {
             if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort)) return false;
             o_free_seen = true;
           }
+          if (!mbar_wait(&bars->v_full[vs], vph, abort)) return false;
           if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort)) return false;
           ++p_use[h];
-          const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
-          const uint32_t s = pos % kKVStages, u = pos / kKVStages;
-          if (!mbar_wait(&bars->v_full[s], u & 1, abort)) return false;
           tc_fence_after();
-          const uint32_t vbase = smem_u32(sm + kOffV + s * kTileBytes);
+          const uint64_t dv = dv0 + uint64_t(vs * kStageDesc);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            mma_ts(tmem + col_o(h), tmem + col_s(h) + k * 8, mnmajor_desc(vbase, k), kIdescPV,
-                   (j == 0 && k == 0) ? 0u : 1u);
-          mma_commit(&bars->v_empty[s]);
+            mma_ts(tmem + col_o(h), tmem + col_s(h) + k * 8, dv + uint64_t(k) * 128u, kIdescPV,
+                   (first && k == 0) ? 0u : 1u);
+          if (++vs == kVStages) { vs = 0; vph ^= 1; }
+          return true;
+        };
+        // S_h = Q K^T for the stream's next block.
+        auto issue_s = [&](int h) -> bool {
+          if (!mbar_wait(&bars->k_full[ks], kph, abort)) return false;
+          const uint64_t dk = dk0 + uint64_t(ks * kStageDesc);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            // step k of the 128-deep contraction: 32 bytes along a 128-byte
+            // swizzled row, then the second 64-column region
+            const uint64_t off = uint64_t((k >> 2) * (kRegionBytes >> 4) + (k & 3) * 2);
+            mma_ss(tmem + col_s(h), dq + off, dk + off, kIdescQK, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&bars->s_full[h]);
+          if (++ks == kKStages) { ks = 0; kph ^= 1; }
           return true;
         };
         if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort))) break;
-        tc_fence_after();
+        // Order per step j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j) -- the load
+        // order of K and of V.  Where stream 1 has one block fewer, its last
+        // PV comes right after S_0 of the extra block, again in load order.
         for (int j = 0; ok && j < t.nb0; ++j) {
-          for (int h = 0; h < 2; ++h) {
-            if (h == 1 && j >= t.nb1) break;
-            if (j > 0 && !(ok = issue_pv(h, j - 1))) break;
-            const uint32_t s = n % kKVStages, u = n / kKVStages;
-            if (!(ok = mbar_wait(&bars->k_full[s], u & 1, abort))) break;
-            tc_fence_after();
-            const uint32_t kbase = smem_u32(sm + kOffK + s * kTileBytes);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              mma_ss(tmem + col_s(h), kmajor_desc(qbase, k), kmajor_desc(kbase, k), kIdescQK,
-                     k > 0 ? 1u : 0u);
-            mma_commit(&bars->s_full[h]);
-            mma_commit(&bars->k_empty[s]);
-            ++n;
+          if (j > 0 && !(ok = issue_pv(0, j == 1))) break;
+          if (!(ok = issue_s(0))) break;
+          if (j < t.nb1) {
+            if (j > 0 && !(ok = issue_pv(1, j == 1))) break;
+            if (!(ok = issue_s(1))) break;
+          } else if (j == t.nb1 && j > 0) {
+            if (!(ok = issue_pv(1, j == 1))) break;
           }
         }
         if (!ok) break;
         mma_commit(&bars->q_empty);  // every S of this unit issued
-        if (!(ok = issue_pv(0, t.nb0 - 1))) break;
-        if (t.nb1 > 0 && !(ok = issue_pv(1, t.nb1 - 1))) break;
+        if (!(ok = issue_pv(0, t.nb0 == 1))) break;
+        if (t.nb1 == t.nb0 && t.nb1 > 0 && !(ok = issue_pv(1, t.nb1 == 1))) break;
         mma_commit(&bars->o_ready);
       }
       // Every MMA issued here completes before TMEM is released.
@@ -292,6 +327,12 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int nv = rows_left < 128 ? int(rows_left) : 128;  // valid keys of the block
         if (!(ok = warp_wait(&bars->s_full[h], use & 1, abort))) break;
         tc_fence_after();
+        if (row == 0) {
+          // S_h(j) is complete, and with it every MMA issued before it: the K
+          // stage it read and the V stage of this stream's previous PV are free.
+          mbar_arrive(&bars->k_empty[(base + uint32_t(seq_pos(t, h, j))) % kKStages]);
+          if (j > 0) mbar_arrive(&bars->v_empty[(base + uint32_t(seq_pos(t, h, j - 1))) % kVStages]);
+        }
         uint32_t sr[128];  // raw fp32 logits of this row
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -361,7 +402,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           // V rows past the valid keys may hold anything (P is 0 there, but
           // 0 * NaN is not 0): zero them before the PV MMA reads the stage.
           const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
-          const uint32_t s = pos % kKVStages, u = pos / kKVStages;
+          const uint32_t s = pos % kVStages, u = pos / kVStages;
           if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort))) break;
           if (row >= nv) {
             uint4* v0 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + row * 128);
@@ -379,10 +420,13 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(&bars->p_full[h]);
       }
       if (!ok) break;
+      // V stage of this stream's last PV (released once both PV chains are done)
+      const uint32_t last_v = mine > 0 ? (base + uint32_t(seq_pos(t, h, mine - 1))) % kVStages : 0u;
       base += uint32_t(t.nb);
       // ---- merge the two streams and write this thread's 64 output columns
       if (!(ok = warp_wait(&bars->o_ready, uc & 1, abort))) break;
       tc_fence_after();
+      if (row == 0 && mine > 0) mbar_arrive(&bars->v_empty[last_v]);
       if (!(ok = warp_wait(&bars->x_read, (uc & 1) ^ 1, abort))) break;  // last unit's reads done
       bars->xml[h][row] = make_float2(m, l);
       mbar_arrive(&bars->x_full);

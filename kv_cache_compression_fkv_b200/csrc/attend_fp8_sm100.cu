@@ -230,57 +230,71 @@ attend_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
+    // One thread issues the MMAs only slightly faster than the tensor core
+    // runs them and the hardware queue is short, so this thread only waits
+    // and issues: ring cursors (K and V are consumed in load order),
+    // precomputed descriptors, one commit per S group (the softmax releases
+    // the K and V stages), a tcgen05 fence only after P and O handoffs.
     if (lane == 0) {
-      uint32_t n = 0, uc = 0;
+      uint32_t uc = 0, ks = 0, kph = 0, vs = 0, vph = 0;
       uint32_t p_use[2] = {0, 0};
       bool ok = true;
-      const uint32_t qbase = smem_u32(sm + kOffQ);
+      const uint64_t dq = kmajor8_desc(smem_u32(sm + kOffQ), 0);
+      const uint64_t dk0 = kmajor8_desc(smem_u32(sm + kOffK), 0);
+      const uint64_t dv0 = mnmajor8_desc(smem_u32(sm + kOffV), 0);
+      constexpr uint32_t kStageDesc = kTile >> 4;  // descriptor step between ring stages
       for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++uc) {
         const Unit t = decode(a, tile);
-        const uint32_t base = n;
         bool o_free_seen = false;
-        auto issue_pv = [&](int h, int j) -> bool {  // O_h += P_h V, stream h's block j
+        // O_h += P_h V for the stream's next block (`first`: its first of the unit).
+        auto issue_pv = [&](int h, bool first) -> bool {
           if (!o_free_seen) {
             if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort)) return false;
             o_free_seen = true;
           }
+          if (!mbar_wait(&bars->v_full[vs], vph, abort)) return false;
           if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort)) return false;
           ++p_use[h];
-          const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
-          const uint32_t s = pos % kStages, u = pos / kStages;
-          if (!mbar_wait(&bars->v_full[s], u & 1, abort)) return false;
           tc_fence_after();
-          const uint32_t vbase = smem_u32(sm + kOffV + s * kTile);
+          // step k: 32 keys = 4 KB further (descriptor address field: bytes >> 4)
+          const uint64_t dv = dv0 + uint64_t(vs * kStageDesc);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_ts_e4m3(tmem + col_o(h), tmem + col_s(h) + k * 8, mnmajor8_desc(vbase, k),
-                        kIdescPV, (j == 0 && k == 0) ? 0u : 1u);
-          mma_commit(&bars->v_empty[s]);
+            mma_ts_e4m3(tmem + col_o(h), tmem + col_s(h) + k * 8, dv + uint64_t(k) * 256u,
+                        kIdescPV, (first && k == 0) ? 0u : 1u);
+          if (++vs == kStages) { vs = 0; vph ^= 1; }
+          return true;
+        };
+        // S_h = Q K^T for the stream's next block; step k: 32 bytes along the row.
+        auto issue_s = [&](int h) -> bool {
+          if (!mbar_wait(&bars->k_full[ks], kph, abort)) return false;
+          const uint64_t dk = dk0 + uint64_t(ks * kStageDesc);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_ss_e4m3(tmem + col_s(h), dq + uint64_t(2 * k), dk + uint64_t(2 * k), kIdescQK,
+                        k > 0 ? 1u : 0u);
+          mma_commit(&bars->s_full[h]);
+          if (++ks == kStages) { ks = 0; kph ^= 1; }
           return true;
         };
         if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort))) break;
-        tc_fence_after();
+        // Per step j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j) -- the load order of K
+        // and of V; where stream 1 has one block fewer, its last PV follows S_0
+        // of the extra block, again in load order.
         for (int j = 0; ok && j < t.nb0; ++j) {
-          for (int h = 0; h < 2; ++h) {
-            if (h == 1 && j >= t.nb1) break;
-            if (j > 0 && !(ok = issue_pv(h, j - 1))) break;
-            const uint32_t s = n % kStages, u = n / kStages;
-            if (!(ok = mbar_wait(&bars->k_full[s], u & 1, abort))) break;
-            tc_fence_after();
-            const uint32_t kbase = smem_u32(sm + kOffK + s * kTile);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma_ss_e4m3(tmem + col_s(h), kmajor8_desc(qbase, k), kmajor8_desc(kbase, k),
-                          kIdescQK, k > 0 ? 1u : 0u);
-            mma_commit(&bars->s_full[h]);
-            mma_commit(&bars->k_empty[s]);
-            ++n;
+          if (j > 0 && !(ok = issue_pv(0, j == 1))) break;
+          if (!(ok = issue_s(0))) break;
+          if (j < t.nb1) {
+            if (j > 0 && !(ok = issue_pv(1, j == 1))) break;
+            if (!(ok = issue_s(1))) break;
+          } else if (j == t.nb1 && j > 0) {
+            if (!(ok = issue_pv(1, j == 1))) break;
           }
         }
         if (!ok) break;
         mma_commit(&bars->q_empty);
-        if (!(ok = issue_pv(0, t.nb0 - 1))) break;
-        if (t.nb1 > 0 && !(ok = issue_pv(1, t.nb1 - 1))) break;
+        if (!(ok = issue_pv(0, t.nb0 == 1))) break;
+        if (t.nb1 == t.nb0 && t.nb1 > 0 && !(ok = issue_pv(1, t.nb1 == 1))) break;
         mma_commit(&bars->o_ready);
       }
       mma_commit(&bars->mma_done);
@@ -333,6 +347,12 @@ attend_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         const float corr0 = svm / sv0, corr1 = svm / sv1;   // >= 1
         const float lsv0 = -__log2f(corr0), lsv1 = -__log2f(corr1);
         if (!(ok = warp_wait(&bars->s_full[h], use & 1, abort))) break;
+        if (row == 0) {
+          // S_h(j) is complete, and with it every MMA issued before it: the K
+          // stage it read and the V stage of this stream's previous PV are free.
+          mbar_arrive(&bars->k_empty[(base + uint32_t(seq_pos(t, h, j))) % kStages]);
+          if (j > 0) mbar_arrive(&bars->v_empty[(base + uint32_t(seq_pos(t, h, j - 1))) % kStages]);
+        }
         tc_fence_after();
         uint32_t sr[128];  // raw fp32 logits of this row (e4m3 codes' dot products)
 #pragma unroll
@@ -433,9 +453,12 @@ attend_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         mbar_arrive(&bars->p_full[h]);
       }
       if (!ok) break;
+      // V stage of this stream's last PV (released once both PV chains are done)
+      const uint32_t last_v = mine > 0 ? (base + uint32_t(seq_pos(t, h, mine - 1))) % kStages : 0u;
       base += uint32_t(t.nb);
       // ---- merge the two streams and write this thread's 64 output columns
       if (!(ok = warp_wait(&bars->o_ready, uc & 1, abort))) break;
+      if (row == 0 && mine > 0) mbar_arrive(&bars->v_empty[last_v]);
       tc_fence_after();
       if (!(ok = warp_wait(&bars->x_read, (uc & 1) ^ 1, abort))) break;  // last unit's reads done
       bars->xml[h][row] = make_float2(m, l);

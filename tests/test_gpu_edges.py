@@ -50,9 +50,11 @@ def test_empty_history(cuda_device):
     parity.check_step(w, x, res)
 
 
-@pytest.mark.parametrize("T,F", [(96, 0), (40, 2), (128, 1)])
+@pytest.mark.parametrize("T,F", [(96, 0), (40, 2), (128, 1), (128, 2)])
 def test_few_key_blocks(cuda_device, T, F):
-    """One or two 128-key blocks in total (one attention stream may be empty)."""
+    """One to three 128-key blocks in total: one attention stream may be
+    empty, or one block shorter than the other (its last PV then follows the
+    other stream's extra S)."""
     w = _small(T=T, F=F, Fc=1, static_frames=tuple(range(F)), k_dynamic=F)
     x = wl.generate(w)
     res = parity.run_step(w, x, comp_rows=max(F * T, 0))

@@ -38,11 +38,11 @@
 //              order, so S_h of block j overwrites P_h only after the PV that
 //              reads it, and by the time S_h is complete the previous PV into
 //              O_h is complete too (the softmax may rescale O_h right away).
-//              The issuing thread is the pace-setter: it issues an M=128,
-//              N=128, K=16 MMA only slightly faster than the tensor core
-//              executes one and the hardware queue is short, so its work
-//              between MMA groups (each mbarrier test or commit costs it
-//              ~90 cycles) is kept to one wait and one commit per group.
+//              The issuing thread issues an M=128, N=128, K=16 MMA only
+//              slightly faster than the tensor core executes one and the
+//              hardware queue is short, so its work between MMA groups (each
+//              mbarrier test or commit costs it ~90 cycles) idles the tensor
+//              core; it is kept to one wait and one commit per group.
 // TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256,384), O_1 [384,512).
 //
 // Key blocks past the valid rows of a range are masked (logit -> -inf) and

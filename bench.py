@@ -17,8 +17,13 @@ events between them.  N > 1: one process per GPU (torchrun), each rank runs
 its own independent chunk step (replicas: the step has no exchange), and the
 time is the max over ranks.
 
+At N = 1 the workloads named by ``--extra`` (default: 1080P, the 30-layer
+480P batch and the 14B token variant) are timed the same way after the
+headline one and reported under ``workloads``.
+
 ``--impl reference`` times the fp64 CPU oracle (the only reference of this
-method) on the host cores, on a bounded sample of the same workload.
+method) on the host cores: each step a bounded sample of whole heads of the
+same workload, ``ms_per_step`` its measured wall time.
 """
 from __future__ import annotations
 
@@ -198,6 +203,107 @@ def max_over_ranks(value, dist=None, device=None):
 def aggregate_throughput(units_per_rank, world, max_ms):
     """Whole-job throughput: units processed by all ranks / slowest rank's time."""
     return units_per_rank * world / (max_ms / 1e3)
+
+
+def kept_per_head(w):
+    """Segments every head keeps in the workload's step: the static mask size
+    (= the dynamic budget k) in frame mode, S + C + R tokens in token mode."""
+    if w.granularity == "token":
+        return int(w.sink_tokens + w.keep_tokens + w.recent_tokens)
+    return int(w.k_dynamic)
+
+
+def bench_config(base, w, world=1, split="replicas", extra=None):
+    """The ``config`` object of the JSON line; both arms print the same one."""
+    cfg = {"workload": base.name, "L": base.L, "H": base.H, "D": w.D, "T": w.T, "F": w.F,
+           "Fc": w.Fc, "granularity": w.granularity, "kept_per_head": kept_per_head(base),
+           "l2": "flushed between timed steps (256 MiB write outside the events)",
+           "parallelism": (f"heads split over {world} GPUs" if split == "heads" and world > 1
+                           else f"replicas x{world}" if world > 1 else "single GPU")}
+    cfg.update(extra or {})
+    return cfg
+
+
+def cpu_model():
+    """Host CPU model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def measure_workload(fkv, w, x_cpu, dev, steps, warmup, flush):
+    """One more workload on this GPU, timed like the headline one: the fused
+    fkv_step (CUDA events around each step, L2 flushed between steps), then the
+    entry points one by one for the per-kernel split and the roofline figures."""
+    p = fkv.params_for(w)
+    stream = torch.cuda.current_stream(dev)
+    x = {k: v.to(dev) for k, v in x_cpu.items()}
+    outs = fkv.allocate(p, dev)
+    io = fkv.make_step_io(p, x, outs)
+    for _ in range(warmup):
+        fkv.step(p, x, outs, io=io)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record(stream)
+        fkv.step(p, x, outs, io=io)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    step_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        e = kev[i]
+        e[0].record(stream)
+        fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
+                           outs["seg_score"], outs["ws"], k_cur=x["k_cur"])
+        e[1].record(stream)
+        fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
+                        x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])
+        e[2].record(stream)
+        fkv.compact_gather(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
+                           outs["k_comp"], outs["v_comp"], outs["ws"])
+        e[3].record(stream)
+        fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"],
+                              outs["v_comp"], outs["kept_cnt"], outs["out"], outs["ws"])
+        e[4].record(stream)
+    torch.cuda.synchronize(dev)
+    st, det = fkv.read_status(outs["ws"])
+    if st != 0:
+        raise RuntimeError(f"device status {st} on head {det} ({w.name})")
+    part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(steps))
+            for j, n in enumerate(["score", "select", "gather", "attend"])}
+    alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
+                      else torch.ones(w.L, w.H))
+    peaks, _ = load_peaks()
+    attn_tfs = alg["attn_flops"] / (part["attend"] * 1e-3) / 1e12
+    gather_gbs = alg["gather_bytes"] / (part["gather"] * 1e-3) / 1e9
+    score = {"ms": round(part["score"], 4)}
+    if alg["score_exps"]:
+        score["frac_sfu"] = round(alg["score_exps"] / (part["score"] * 1e-3) / SFU_EXP2_PER_S, 4)
+    else:
+        score["frac_hbm"] = round(alg["score_bytes"] / (part["score"] * 1e-3) / 1e9
+                                  / peaks["hbm_gbs"], 4)
+    res = {"value": round(aggregate_throughput(w.L * steps, 1, step_ms * steps), 3), "unit": UNIT,
+           "ms_per_step": round(step_ms, 4), "steps": steps, "warmup": warmup,
+           "config": bench_config(w, w),
+           "kernels": {"score_segments": score, "select_topk": {"ms": round(part["select"], 4)},
+                       "compact_gather": {"ms": round(part["gather"], 4),
+                                          "GB/s": round(gather_gbs, 1),
+                                          "frac_hbm": round(gather_gbs / peaks["hbm_gbs"], 4)},
+                       "attend_compressed": {"ms": round(part["attend"], 4),
+                                             "TFLOP/s": round(attn_tfs, 2),
+                                             "frac_tensor": round(attn_tfs / peaks["bf16_tflops"], 4)}}}
+    del x, outs, io
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_ours(args, rank, world, local_rank):
@@ -507,14 +613,10 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "strong" if args.split == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "fp32", "data": "synthetic (seeded, Wan-shaped)",
-        "config": {"workload": base.name, "L": base.L, "H": base.H, "D": w.D, "T": w.T, "F": w.F,
-                   "Fc": w.Fc, "granularity": w.granularity,
-                   "kept_per_head": int(outs["kept_cnt"][0, 0]),
-                   "l2": "flushed between timed steps (256 MiB write outside the events)",
-                   "parallelism": (f"heads split over {world} GPUs" if args.split == "heads" and world > 1
-                                   else f"replicas x{world}" if world > 1 else "single GPU"),
-                   **({"heads_per_rank": f"{w.H} (rank {rank})", "gather_out_ms": round(gather_ms, 4)}
-                      if gather_ms is not None else {})},
+        "config": bench_config(base, w, world, args.split,
+                               {"heads_per_rank": f"{w.H} (rank {rank})",
+                                "gather_out_ms": round(gather_ms, 4)} if gather_ms is not None
+                               else None),
         "impl": "ours",
         "e2e": {"value": round(e2e_value, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -553,6 +655,17 @@ def run_ours(args, rank, world, local_rank):
                                               kernel_source_hash(_attend_fp8_sources()))},
             },
         }
+    extra = [n for n in args.extra.split(",") if n and n != base.name] if world == 1 else []
+    if extra:
+        # the metric's other resolution and the other configurations, timed on the
+        # same GPU after the headline workload (inputs generated outside the timing)
+        line["workloads"] = {}
+        with ClockSampler(local_rank) as clk_x:
+            for name in extra:
+                we = wl.get(name)
+                line["workloads"][name] = measure_workload(
+                    fkv, we, wl.generate(we), dev, min(args.steps, 10), args.warmup, flush)
+        line["workloads_clocks"] = clk_x.summary()
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget)
     if dist is not None:
@@ -573,65 +686,97 @@ def _attend_fp8_sources():
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(w, x_cpu, budget_s=15.0):
-    """Times the fp64 oracle, as it stands, on a bounded sample: whole heads
-    (scoring, selection, compaction, attention over every query row) taken in
-    order until the budget is spent; value scaled to layer-steps per second."""
+def _oracle_head(w, x, l, h):
+    """One (layer, head) of the step through the fp64 oracle, as it stands:
+    scoring and selection, compaction, attention over every query row."""
     from oracle import fkv_oracle as orc
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    x = {k: v for k, v in x_cpu.items()}
-    heads_done, t0 = 0, time.perf_counter()
+    f64 = lambda k: wl.as_float64(x[k][l, h])  # noqa: E731
+    ks, _ = orc.head_keep(
+        granularity=w.granularity,
+        dynamic=w.granularity == "token" or bool(x["head_role"][l, h]),
+        mask_row=x["static_mask"][l, h].numpy(), k=int(x["k_per_head"][l, h]),
+        q_cur=f64("q_cur"), k_hist=f64("k_hist"), T=w.T, scale=w.scale,
+        score_stride=w.score_stride, q_score=f64("q_score") if "q_score" in x else None,
+        sink=w.sink_tokens, recent=w.recent_tokens,
+        k_chunk=f64("k_cur") if w.score_with_chunk else None,
+        token_static_mask=w.static_token_mask)
+    seg_len = w.T if (w.granularity == "frame" and not w.static_token_mask) else 1
+    keys = np.concatenate([orc.compact(f64("k_hist"), ks, seg_len), f64("k_cur")])
+    vals = np.concatenate([orc.compact(f64("v_hist"), ks, seg_len), f64("v_cur")])
+    orc.attention(f64("q_cur"), keys, vals, w.scale)
+
+
+def _head_order(w, x):
+    """(layer, head) pairs alternating dynamic and static heads, so that any
+    prefix of the order has the layer's mix of the two."""
     order = [(l, h) for l in range(w.L) for h in range(w.H)]
-    # alternate static / dynamic heads so the sample has the mix of the layer
     if w.granularity == "frame":
         role = x["head_role"]
         dyn = [lh for lh in order if role[lh]]
         sta = [lh for lh in order if not role[lh]]
         order = [v for pair in zip(dyn, sta) for v in pair] + dyn[len(sta):] + sta[len(dyn):]
-    for (l, h) in order:
-        f64 = lambda k: wl.as_float64(x[k][l, h])  # noqa: E731
-        ks, _ = orc.head_keep(
-            granularity=w.granularity,
-            dynamic=w.granularity == "token" or bool(x["head_role"][l, h]),
-            mask_row=x["static_mask"][l, h].numpy(), k=int(x["k_per_head"][l, h]),
-            q_cur=f64("q_cur"), k_hist=f64("k_hist"), T=w.T, scale=w.scale,
-            score_stride=w.score_stride, q_score=f64("q_score") if "q_score" in x else None,
-            sink=w.sink_tokens, recent=w.recent_tokens,
-            k_chunk=f64("k_cur") if w.score_with_chunk else None,
-            token_static_mask=w.static_token_mask)
-        seg_len = w.T if (w.granularity == "frame" and not w.static_token_mask) else 1
-        keys = np.concatenate([orc.compact(f64("k_hist"), ks, seg_len), f64("k_cur")])
-        vals = np.concatenate([orc.compact(f64("v_hist"), ks, seg_len), f64("v_cur")])
-        orc.attention(f64("q_cur"), keys, vals, w.scale)
+    return order
+
+
+def _cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
+def cpu_baseline(w, x_cpu, budget_s=15.0):
+    """Times the fp64 oracle, as it stands, on a bounded sample: whole heads
+    (scoring, selection, compaction, attention over every query row) taken in
+    order until the budget is spent; value scaled to layer-steps per second."""
+    heads_done, t0 = 0, time.perf_counter()
+    for (l, h) in _head_order(w, x_cpu):
+        _oracle_head(w, x_cpu, l, h)
         heads_done += 1
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
     layers = heads_done / w.H
-    return {"value": round(layers / dt, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+    return {"value": round(layers / dt, 6), "unit": UNIT, "cores": _cores(),
+            "cpu_model": cpu_model(), "kind": "oracle",
             "sample": f"{heads_done} of {w.L * w.H} heads of workload {w.name} (full oracle step "
                       f"per head, every query row), {dt:.1f} s, numpy fp64",
             "seconds": round(dt, 2)}
 
 
 def run_reference(args):
+    """The reference arm: the fp64 oracle, as it stands, on the host cores.
+    One "step" is a bounded sample of the workload's chunk step: a fixed number
+    of whole heads (one dynamic and one static head by default, every query
+    row), taken in turn from the layer's alternating order so that successive
+    steps walk through all of its heads.  ``ms_per_step`` is the measured wall
+    time of such a step; ``value`` = the layers these steps covered (heads / H)
+    per second of their total time."""
     w = wl.get(args.workload)
     x_cpu = wl.generate(w)
-    vals = []
+    order = _head_order(w, x_cpu)
+    per_step = max(1, min(args.ref_heads, len(order)))
+    pos, times = 0, []
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget / max(1, args.steps))
+        t0 = time.perf_counter()
+        for _ in range(per_step):
+            l, h = order[pos % len(order)]
+            _oracle_head(w, x_cpu, l, h)
+            pos += 1
+        dt = time.perf_counter() - t0
         if i >= args.warmup:
-            vals.append(r)
-    value = statistics.mean(v["value"] for v in vals)
-    cb = dict(vals[-1])
-    cb["value"] = round(value, 6)
+            times.append(dt)
+    total_s = sum(times)
+    value = (per_step * args.steps / w.H) / total_s
+    cb = {"value": round(value, 6), "unit": UNIT, "cores": _cores(), "cpu_model": cpu_model(),
+          "kind": "oracle",
+          "sample": f"{per_step} of {w.L * w.H} heads of workload {w.name} per step (full oracle "
+                    f"step per head, every query row), {args.steps} timed steps in "
+                    f"{total_s:.1f} s, numpy fp64",
+          "seconds": round(total_s, 2)}
     return {
         "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3) if value else None,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * total_s / args.steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded, Wan-shaped)",
-        "config": {"workload": w.name, "L": w.L, "H": w.H, "D": w.D, "T": w.T, "F": w.F, "Fc": w.Fc,
-                   "granularity": w.granularity},
+        "config": bench_config(w, w),
         "impl": "reference", "cpu_baseline": cb,
         "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -648,7 +793,12 @@ def main():
                     help="N > 1: independent replicas per GPU (weak scaling) or the heads of "
                          "one step split across GPUs (strong scaling)")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-heads", type=int, default=2,
+                    help="reference arm: whole heads of the workload per timed step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra", default="1080p,480p_30layer,token14b",
+                    help="N = 1: further workloads timed after the headline one, reported "
+                         "under 'workloads' (empty string: none)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     rank = int(os.environ.get("RANK", "0"))

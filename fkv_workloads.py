@@ -275,9 +275,22 @@ def sample_rows(n_rows: int, n_samples: int, seed: int) -> np.ndarray:
     return np.unique(np.concatenate([pick, [0, n_rows - 1]]))
 
 
+def tile_rows(n_rows: int, seed: int, tile: int = 128, per_tile: int = 1) -> np.ndarray:
+    """Sorted distinct query rows with ``per_tile`` random rows inside every
+    ``tile``-row block (the last, ragged block included) plus the first and the
+    last row, so that every query tile of a head is checked."""
+    rng = np.random.default_rng(seed)
+    picks = [np.array([0, n_rows - 1])]
+    for start in range(0, n_rows, tile):
+        stop = min(n_rows, start + tile)
+        picks.append(rng.choice(np.arange(start, stop), size=min(per_tile, stop - start),
+                                replace=False))
+    return np.unique(np.concatenate(picks))
+
+
 __all__: Sequence[str] = (
     "Workload", "WORKLOADS", "STATIC_FRAMES_18", "get", "scaled", "generate",
-    "as_float64", "sample_rows",
+    "as_float64", "sample_rows", "tile_rows",
 )
 
 

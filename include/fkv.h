@@ -54,8 +54,9 @@ extern "C" {
 #endif
 
 /* 3: adds fkv_fp8_cache_t and the three *_fp8 entry points;
- * 4: adds fkv_select_heuristic; 5: adds fkv_step_fp8. */
-#define FKV_ABI_VERSION 5
+ * 4: adds fkv_select_heuristic; 5: adds fkv_step_fp8;
+ * 6: adds fkv_diag_attend_timeout. */
+#define FKV_ABI_VERSION 6
 
 typedef enum fkv_status {
   FKV_OK = 0,
@@ -175,6 +176,23 @@ int32_t fkv_step_launches(const fkv_params_t* p, int32_t* launches);
  * device arrays of n floats. */
 int32_t fkv_exp2_emulated(const float* x, float* y, int64_t n, void* stream);
 
+/* Diagnostic of the failure path: fkv_attend_compressed (bf16 tensor-core
+ * kernel) with every bounded device wait limited to wait_cycles SM cycles
+ * (10^4 .. 2*10^9; production calls use 2*10^9, about one second) and with
+ * CTA 0 withholding the completion signal of its first logit tile, so that
+ * the softmax's wait for it runs out.  The MMAs behind the signal are issued
+ * and complete; nothing else is left outstanding.  Expected result: the call
+ * returns FKV_OK, every CTA winds down (waiting, bounded, for its own copies
+ * and MMAs, then freeing its tensor memory), and fkv_read_status reports
+ * FKV_ERR_TIMEOUT with detail 0 (the CTA that gave up); `out` rows of the
+ * work units CTA 0 owned are left unwritten, the other rows are the
+ * attention.  No trap, no fault: the context stays usable.  fp32 params:
+ * FKV_ERR_UNSUPPORTED. */
+int32_t fkv_diag_attend_timeout(const fkv_params_t* p, const void* q_cur, const void* k_cur,
+                                const void* v_cur, const void* k_comp, const void* v_comp,
+                                const int32_t* kept_cnt, void* out, int64_t wait_cycles, void* ws,
+                                void* stream);
+
 /* Zeroes the workspace (status word included) on `stream`.  Call once after
  * allocating it; entry points never clear the status word themselves. */
 int32_t fkv_workspace_init(void* ws, size_t bytes, void* stream);
@@ -211,14 +229,20 @@ int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void*
  * 480P batch) are rejected with FKV_ERR_WORKSPACE and nothing is launched.  It calls no
  * cudaMalloc / cudaFree.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make
- *    that first call before any stream capture.
+ *    (cudaGetSymbolAddress, with that device current) and caches it for the
+ *    life of the process; make that first call before any stream capture.
+ *    The cached address belongs to the device's current CUDA context: after
+ *    cudaDeviceReset (or anything else that destroys that context) it is
+ *    stale, so do not call this entry point on a device after resetting it.
  *  - Every call on a device shares the one array and leaves its contents
- *    behind; nothing in it has to start at zero (every partial statistic is
- *    written before it is read).  Calls that overlap on the GPU (different
- *    streams, or threads) race on it and must be serialised by the caller.
- *  - Device-side errors of this call are not reported (there is no workspace
- *    status word for the caller to read). */
+ *    behind.  Each call first clears the 256-byte status block at the start
+ *    of the array (a cudaMemsetAsync on `stream`); the partial statistics
+ *    after it are written before they are read and need no clearing.  Calls
+ *    that overlap on the GPU (different streams, or threads) race on the
+ *    array and must be serialised by the caller.
+ *  - There is no status word for the caller to read: a device-side failure
+ *    of the scoring (a bounded wait that gave up) instead makes every dynamic
+ *    head's scores NaN. */
 int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void* q_cur, const void* q_score,
                                    const void* k_hist, const void* k_cur,
                                    const uint8_t* head_role, float* seg_score, void* stream);

@@ -42,8 +42,9 @@ __device__ __forceinline__ int seq_pos(const Unit& t, int h, int j) {
 // Key block index of (stream h, j).
 __device__ __forceinline__ int block_of(const Unit& t, int h, int j) { return h ? t.nb0 + j : j; }
 
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  const bool ok = mbar_wait(bar, parity, abort);
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long limit = kWaitCycles) {
+  const bool ok = mbar_wait(bar, parity, abort, limit);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -84,6 +84,7 @@ constexpr int kMmaWarp = 9;
 constexpr uint32_t kIdescQK = idesc_bf16(128, 128, false);
 constexpr uint32_t kIdescPV = idesc_bf16(128, 128, true);
 constexpr float kRescaleLog2 = 8.0f;
+static_assert(kProductionWaitCycles == kWaitCycles, "one production wait limit");
 // One of every FKV_POLY_EVERY exponential pairs goes to the FMA-pipe exp2 (0: none).
 #ifndef FKV_POLY_EVERY
 #define FKV_POLY_EVERY 0
@@ -122,6 +123,9 @@ struct AttnArgs {
   const int32_t* kept_cnt;
   __nv_bfloat16* out;
   int32_t* status;
+  long long wait_cycles;  // limit of every bounded wait (kWaitCycles in production)
+  int withhold_s0;        // diagnostic: CTA 0 withholds the completion signal of its
+                          // first S_0 group (0 in production)
 };
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -182,7 +186,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x) {
         const Unit t = decode(a, tile);
-        if (!(ok = mbar_wait(&bars->q_empty, (tc & 1) ^ 1, abort))) break;
+        if (!(ok = mbar_wait(&bars->q_empty, (tc & 1) ^ 1, abort, a.wait_cycles))) break;
         mbar_expect_tx(&bars->q_full, kTileBytes);
         tma_load_tile(sm + kOffQ, &tm_q, &bars->q_full, t.qt * 128, t.lh);
         ++tc;
@@ -193,7 +197,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const bool inA = b < t.nbA;
             const int row = (inA ? b : b - t.nbA) * 128;
             const uint32_t s = n % kKStages, u = n / kKStages;
-            if (!(ok = mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort))) break;
+            if (!(ok = mbar_wait(&bars->k_empty[s], (u & 1) ^ 1, abort, a.wait_cycles))) break;
             mbar_expect_tx(&bars->k_full[s], kTileBytes);
             tma_load_tile(sm + kOffK + s * kTileBytes, inA ? &tm_kc : &tm_kn, &bars->k_full[s],
                           row, t.lh);
@@ -218,7 +222,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const bool inA = b < t.nbA;
             const int row = (inA ? b : b - t.nbA) * 128;
             const uint32_t s = n % kVStages, u = n / kVStages;
-            if (!(ok = mbar_wait(&bars->v_empty[s], (u & 1) ^ 1, abort))) break;
+            if (!(ok = mbar_wait(&bars->v_empty[s], (u & 1) ^ 1, abort, a.wait_cycles))) break;
             mbar_expect_tx(&bars->v_full[s], kTileBytes);
             tma_load_tile(sm + kOffV + s * kTileBytes, inA ? &tm_vc : &tm_vn, &bars->v_full[s],
                           row, t.lh);
@@ -242,6 +246,10 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t uc = 0, ks = 0, kph = 0, vs = 0, vph = 0;
       uint32_t p_use[2] = {0, 0};
       bool ok = true;
+      // Diagnostic only: one software arrival that never comes, so that the
+      // softmax's bounded wait on it runs out (the MMAs themselves are issued
+      // and complete; nothing else is left outstanding behind the signal).
+      bool withhold = a.withhold_s0 != 0 && blockIdx.x == 0;
       const uint64_t dq = kmajor_desc(smem_u32(sm + kOffQ), 0);
       const uint64_t dk0 = kmajor_desc(smem_u32(sm + kOffK), 0);
       const uint64_t dv0 = mnmajor_desc(smem_u32(sm + kOffV), 0);
@@ -252,11 +260,11 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         // O_h += P_h V for the stream's next block (`first`: its first of the unit).
         auto issue_pv = [&](int h, bool first) -> bool {
           if (!o_free_seen) {
-            if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort)) return false;
+            if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort, a.wait_cycles)) return false;
             o_free_seen = true;
           }
-          if (!mbar_wait(&bars->v_full[vs], vph, abort)) return false;
-          if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort)) return false;
+          if (!mbar_wait(&bars->v_full[vs], vph, abort, a.wait_cycles)) return false;
+          if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort, a.wait_cycles)) return false;
           ++p_use[h];
           tc_fence_after();
           const uint64_t dv = dv0 + uint64_t(vs * kStageDesc);
@@ -269,7 +277,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         };
         // S_h = Q K^T for the stream's next block.
         auto issue_s = [&](int h) -> bool {
-          if (!mbar_wait(&bars->k_full[ks], kph, abort)) return false;
+          if (!mbar_wait(&bars->k_full[ks], kph, abort, a.wait_cycles)) return false;
           const uint64_t dk = dk0 + uint64_t(ks * kStageDesc);
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
@@ -278,11 +286,12 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
             const uint64_t off = uint64_t((k >> 2) * (kRegionBytes >> 4) + (k & 3) * 2);
             mma_ss(tmem + col_s(h), dq + off, dk + off, kIdescQK, k > 0 ? 1u : 0u);
           }
-          mma_commit(&bars->s_full[h]);
+          if (withhold && h == 0) withhold = false;
+          else mma_commit(&bars->s_full[h]);
           if (++ks == kKStages) { ks = 0; kph ^= 1; }
           return true;
         };
-        if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort))) break;
+        if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort, a.wait_cycles))) break;
         // Order per step j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j) -- the load
         // order of K and of V.  Where stream 1 has one block fewer, its last
         // PV comes right after S_0 of the extra block, again in load order.
@@ -325,7 +334,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const bool inA = b < t.nbA;
         const int64_t rows_left = (inA ? t.nA : a.Lq) - int64_t(inA ? b : b - t.nbA) * 128;
         const int nv = rows_left < 128 ? int(rows_left) : 128;  // valid keys of the block
-        if (!(ok = warp_wait(&bars->s_full[h], use & 1, abort))) break;
+        if (!(ok = warp_wait(&bars->s_full[h], use & 1, abort, a.wait_cycles))) break;
         tc_fence_after();
         if (row == 0) {
           // S_h(j) is complete, and with it every MMA issued before it: the K
@@ -403,7 +412,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           // 0 * NaN is not 0): zero them before the PV MMA reads the stage.
           const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
           const uint32_t s = pos % kVStages, u = pos / kVStages;
-          if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort))) break;
+          if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort, a.wait_cycles))) break;
           if (row >= nv) {
             uint4* v0 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + row * 128);
             uint4* v1 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + kRegionBytes + row * 128);
@@ -424,13 +433,13 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint32_t last_v = mine > 0 ? (base + uint32_t(seq_pos(t, h, mine - 1))) % kVStages : 0u;
       base += uint32_t(t.nb);
       // ---- merge the two streams and write this thread's 64 output columns
-      if (!(ok = warp_wait(&bars->o_ready, uc & 1, abort))) break;
+      if (!(ok = warp_wait(&bars->o_ready, uc & 1, abort, a.wait_cycles))) break;
       tc_fence_after();
       if (row == 0 && mine > 0) mbar_arrive(&bars->v_empty[last_v]);
-      if (!(ok = warp_wait(&bars->x_read, (uc & 1) ^ 1, abort))) break;  // last unit's reads done
+      if (!(ok = warp_wait(&bars->x_read, (uc & 1) ^ 1, abort, a.wait_cycles))) break;  // last unit's reads done
       bars->xml[h][row] = make_float2(m, l);
       mbar_arrive(&bars->x_full);
-      if (!(ok = warp_wait(&bars->x_full, uc & 1, abort))) break;
+      if (!(ok = warp_wait(&bars->x_full, uc & 1, abort, a.wait_cycles))) break;
       const float2 other = bars->xml[h ^ 1][row];
       mbar_arrive(&bars->x_read);
       const float m0 = h ? other.x : m, l0 = h ? other.y : l;
@@ -497,7 +506,7 @@ __global__ void exp2_poly_kernel(const float* __restrict__ x, float* __restrict_
 cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_cur,
                                 const void* v_cur, const void* k_comp, const void* v_comp,
                                 const int32_t* kept_cnt, void* out, int32_t* status,
-                                cudaStream_t s) {
+                                cudaStream_t s, long long wait_cycles, bool withhold_s0) {
   using namespace sm100;
   const uint64_t row_b = 128 * 2;
   CUtensorMap tq, tkc, tvc, tkn, tvn;
@@ -525,6 +534,8 @@ cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_
   a.kept_cnt = kept_cnt;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.status = status;
+  a.wait_cycles = wait_cycles;
+  a.withhold_s0 = withhold_s0 ? 1 : 0;
   cudaError_t e = cudaFuncSetAttribute(attend_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmem));
   if (e != cudaSuccess) return e;

@@ -119,7 +119,7 @@ static char* ws_at(void* ws, size_t off) { return reinterpret_cast<char*>(ws) + 
 
 static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, const void* k_hist,
                         const void* k_cur, const uint8_t* head_role, float* seg_score, void* ws,
-                        cudaStream_t s) {
+                        cudaStream_t s, bool poison_on_error = false) {
   WsLayout w = ws_layout(d);
   if (d.token) {
     if (d.nseg == 0) return FKV_OK;
@@ -135,8 +135,9 @@ static int32_t do_score(const Dims& d, const void* q_cur, const void* q_score, c
                                                     status_ptr(ws), s)
                          : launch_score_frame_simt(d, q_cur, k_hist, k_cur, head_role, part, s);
   if (e != cudaSuccess) return cuda_status(e);
-  return cuda_status(
-      launch_score_frame_finalize(d, score_layout(d), head_role, part, rows, seg_score, s));
+  return cuda_status(launch_score_frame_finalize(d, score_layout(d), head_role, part, rows,
+                                                 seg_score, s,
+                                                 poison_on_error ? status_ptr(ws) : nullptr));
 }
 
 static int32_t do_select(const Dims& d, const float* seg_score, const uint8_t* head_role,
@@ -278,6 +279,16 @@ int32_t fkv_read_status(const void* ws, void* stream, int32_t* device_status, in
 int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void* q_score,
                            const void* k_hist, const void* k_cur, const uint8_t* head_role,
                            float* seg_score, void* ws, void* stream) {
+  return fkv::score_segments_checked(p, q_cur, q_score, k_hist, k_cur, head_role, seg_score, ws,
+                                     stream, false);
+}
+
+}  // extern "C"
+
+int32_t fkv::score_segments_checked(const fkv_params_t* p, const void* q_cur,
+                                    const void* q_score, const void* k_hist, const void* k_cur,
+                                    const uint8_t* head_role, float* seg_score, void* ws,
+                                    void* stream, bool poison_on_error) {
   Dims d;
   int32_t st = make_dims(p, &d);
   if (st != FKV_OK) return st;
@@ -293,8 +304,10 @@ int32_t fkv_score_segments(const fkv_params_t* p, const void* q_cur, const void*
   if (d.score_with_chunk && (!k_cur || !aligned16(k_cur))) return FKV_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws)) != FKV_OK) return st;
   return do_score(d, q_cur, q_score, k_hist, k_cur, head_role, seg_score, ws,
-                  static_cast<cudaStream_t>(stream));
+                  static_cast<cudaStream_t>(stream), poison_on_error);
 }
+
+extern "C" {
 
 int32_t fkv_select_topk(const fkv_params_t* p, const float* seg_score, const uint8_t* head_role,
                         const uint8_t* static_mask, const int32_t* k_per_head, int32_t* kept_idx,
@@ -340,6 +353,26 @@ int32_t fkv_attend_compressed(const fkv_params_t* p, const void* q_cur, const vo
   if ((st = check_ws(d, ws)) != FKV_OK) return st;
   return do_attend(d, q_cur, k_cur, v_cur, k_comp, v_comp, kept_cnt, out, ws,
                    static_cast<cudaStream_t>(stream));
+}
+
+int32_t fkv_diag_attend_timeout(const fkv_params_t* p, const void* q_cur, const void* k_cur,
+                                const void* v_cur, const void* k_comp, const void* v_comp,
+                                const int32_t* kept_cnt, void* out, int64_t wait_cycles, void* ws,
+                                void* stream) {
+  Dims d;
+  int32_t st = make_dims(p, &d);
+  if (st != FKV_OK) return st;
+  if (!d.bf16) return FKV_ERR_UNSUPPORTED;  // the tensor-core kernel's waits
+  if (wait_cycles < 10000 || wait_cycles > kProductionWaitCycles) return FKV_ERR_SHAPE;
+  if (!q_cur || !k_cur || !v_cur || ((!k_comp || !v_comp) && d.comp_rows > 0) || !kept_cnt || !out)
+    return FKV_ERR_INVALID_ARG;
+  if (!aligned16(q_cur) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(k_comp) ||
+      !aligned16(v_comp) || !aligned16(out))
+    return FKV_ERR_INVALID_ARG;
+  if ((st = check_ws(d, ws)) != FKV_OK) return st;
+  return cuda_status(launch_attend_sm100(d, q_cur, k_cur, v_cur, k_comp, v_comp, kept_cnt, out,
+                                         status_ptr(ws), static_cast<cudaStream_t>(stream),
+                                         wait_cycles, true));
 }
 
 int32_t fkv_compact_gather_rope(const fkv_params_t* p, const void* k_hist, const void* v_hist,

@@ -96,10 +96,18 @@ cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void
                                     cudaStream_t s);
 // part_ml has the layout of score_layout(d), [head][n_s rows][E entries]; the
 // finalize overwrites the m of each frame's first entry with that frame's
-// per-row mass.
+// per-row mass.  poison (nullable): a status word; when it is nonzero at the
+// finalize, every dynamic head's scores are written NaN.
 cudaError_t launch_score_frame_finalize(const Dims& d, const ScoreLayout& sl,
                                         const uint8_t* head_role, float2* part_ml,
-                                        float2* row_ml, float* seg_score, cudaStream_t s);
+                                        float2* row_ml, float* seg_score, cudaStream_t s,
+                                        const int32_t* poison = nullptr);
+// fkv_score_segments after its host-side checks; poison_on_error: scores of
+// dynamic heads come out NaN when the workspace status word is nonzero by the
+// time the scores are summed (used where the caller cannot read the status).
+int32_t score_segments_checked(const fkv_params_t* p, const void* q_cur, const void* q_score,
+                               const void* k_hist, const void* k_cur, const uint8_t* head_role,
+                               float* seg_score, void* ws, void* stream, bool poison_on_error);
 cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k_hist,
                                float* qbar, float* seg_score, cudaStream_t s);
 cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uint8_t* head_role,
@@ -119,10 +127,14 @@ cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
 cudaError_t launch_score_frame_sm100(const Dims& d, const void* q_cur, const void* k_hist,
                                      const void* k_cur, const uint8_t* head_role, float2* part_ml,
                                      int32_t* status, cudaStream_t s);
+// wait_cycles bounds every mbarrier wait; withhold_s0 (diagnostic) makes CTA 0
+// withhold one completion signal so that a wait runs out.
+constexpr long long kProductionWaitCycles = 2000000000LL;
 cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_cur,
                                 const void* v_cur, const void* k_comp, const void* v_comp,
                                 const int32_t* kept_cnt, void* out, int32_t* status,
-                                cudaStream_t s);
+                                cudaStream_t s, long long wait_cycles = kProductionWaitCycles,
+                                bool withhold_s0 = false);
 cudaError_t launch_gather_rope(const Dims& d, const void* k_hist, const void* v_hist,
                                const int32_t* kept_idx, const int32_t* kept_cnt,
                                const float* omega, int32_t n_pairs, void* k_comp, void* v_comp,

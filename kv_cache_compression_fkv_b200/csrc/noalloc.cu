@@ -83,15 +83,19 @@ extern "C" int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void*
   void* scratch = fkv::scratch_address(&st);
   if (!scratch) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The status block at the start of the scratch must read zero when the
-  // kernels start; the partial statistics are fully written before use.
+  // The status block at the start of the scratch is cleared on every call, so
+  // that a failure recorded by an earlier call does not mark this one; the
+  // partial statistics after it are fully written before they are read.
   cudaError_t e = cudaMemsetAsync(scratch, 0, 256, s);
   if (e != cudaSuccess) {
     fprintf(stderr, "fkv_score_segments_noalloc: %s\n", cudaGetErrorString(e));
     return FKV_ERR_CUDA;
   }
   // Same validation and kernels as fkv_score_segments, with the static array
-  // (256-byte aligned, large enough as checked above) as the workspace.
-  return fkv_score_segments(p, q_cur, q_score, k_hist, k_cur, head_role, seg_score, scratch,
-                            stream);
+  // (256-byte aligned, large enough as checked above) as the workspace.  The
+  // caller has no status word to read, so a device-side failure of the
+  // scoring (a bounded wait that gave up) turns the dynamic heads' scores
+  // into NaN instead of leaving stale values behind.
+  return fkv::score_segments_checked(p, q_cur, q_score, k_hist, k_cur, head_role, seg_score,
+                                     scratch, stream, true);
 }

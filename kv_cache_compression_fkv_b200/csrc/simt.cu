@@ -181,12 +181,17 @@ constexpr int kFrameThreads = 256;
 
 __global__ void __launch_bounds__(kFrameThreads)
 score_frames_kernel(int F, int split, int E, int64_t n_s, const uint8_t* __restrict__ head_role,
-                    const float2* __restrict__ part_ml, float* __restrict__ seg_score) {
+                    const float2* __restrict__ part_ml, float* __restrict__ seg_score,
+                    const int32_t* __restrict__ poison) {
   __shared__ float wsum[kFrameThreads / 32];
   const int f = blockIdx.x, lh = blockIdx.y;
   float* out = seg_score + int64_t(lh) * F + f;
   if (!head_role[lh]) {
     if (threadIdx.x == 0) *out = 0.f;
+    return;
+  }
+  if (poison && *poison != 0) {  // the statistics kernel gave up: no score to give
+    if (threadIdx.x == 0) *out = __int_as_float(0x7fc00000);  // NaN
     return;
   }
   const float2* cf = part_ml + int64_t(lh) * n_s * E + f * split;
@@ -225,7 +230,8 @@ cudaError_t launch_score_frame_simt(const Dims& d, const void* q_cur, const void
 
 cudaError_t launch_score_frame_finalize(const Dims& d, const ScoreLayout& sl,
                                         const uint8_t* head_role, float2* part_ml,
-                                        float2* row_ml, float* seg_score, cudaStream_t s) {
+                                        float2* row_ml, float* seg_score, cudaStream_t s,
+                                        const int32_t* poison) {
   if (d.n_s > 0) {
     dim3 grid(unsigned((d.n_s + kRowWarps - 1) / kRowWarps), unsigned(d.LH));
     score_rows_kernel<<<grid, kRowWarps * 32, 0, s>>>(d.F, sl.split, sl.chunk, sl.E, d.n_s,
@@ -235,7 +241,7 @@ cudaError_t launch_score_frame_finalize(const Dims& d, const ScoreLayout& sl,
   }
   if (d.F < 1) return cudaSuccess;
   score_frames_kernel<<<dim3(unsigned(d.F), unsigned(d.LH)), kFrameThreads, 0, s>>>(
-      d.F, sl.split, sl.E, d.n_s, head_role, part_ml, seg_score);
+      d.F, sl.split, sl.E, d.n_s, head_role, part_ml, seg_score, poison);
   return cudaGetLastError();
 }
 

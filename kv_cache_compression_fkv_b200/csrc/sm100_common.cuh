@@ -79,16 +79,18 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase of the given parity to complete.  Gives up (returns
-// false) when *abort is set by another thread or after kWaitCycles, in which
-// case it sets *abort itself so that every role of the CTA winds down.  A
-// phase that has already completed is seen by a non-blocking test.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// false) when *abort is set by another thread or after `limit` cycles (by
+// default kWaitCycles), in which case it sets *abort itself so that every
+// role of the CTA winds down.  A phase that has already completed is seen by
+// a non-blocking test.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long limit = kWaitCycles) {
   if (mbar_test_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
       return false;
     }

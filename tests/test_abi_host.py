@@ -97,7 +97,7 @@ def test_fp8_entry_points_validate_before_launch(lib):
 
 
 def test_status_strings_and_version(lib):
-    assert lib.fkv_abi_version() == 5
+    assert lib.fkv_abi_version() == 6
     for code in range(8):
         assert lib.fkv_status_string(code).decode().startswith("FKV_")
     assert lib.fkv_status_string(99) == b"FKV_ERR_UNKNOWN"

@@ -6,6 +6,7 @@ import json
 import os
 import subprocess
 import sys
+import time
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -13,9 +14,11 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def _run(env_extra):
     env = dict(os.environ)
     env.update(env_extra)
+    t0 = time.perf_counter()
     r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload", "tiny",
                         "--steps", "3", "--warmup", "3"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    r.wall_s = time.perf_counter() - t0
     return r
 
 
@@ -36,8 +39,17 @@ def test_reference_arm_line():
     assert d["vs_baseline"] is None
     assert d["dtype"] == "f64"
     assert d["config"]["workload"] == "tiny"
+    # the same config object as the GPU arm prints for this workload
+    sys.path.insert(0, ROOT)
+    import bench
+    import fkv_workloads as wl
+    w = wl.get("tiny")
+    assert d["config"] == bench.bench_config(w, w)
+    # the timed steps fit inside the process's own wall time
+    assert d["steps"] * d["ms_per_step"] / 1e3 <= r.wall_s
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert "cpu_model" in cb
     assert cb["unit"] == d["unit"] and isinstance(cb["sample"], str) and cb["sample"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]

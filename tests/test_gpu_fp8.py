@@ -189,3 +189,40 @@ def test_attend_fp8_1080p_sampled_rows(cuda_device):
         ref, tol = _oracle_fp8_attention(x, w, l, h, kept, rows)
         got = out[l, h, rows].cpu().double().numpy()
         assert np.all(np.abs(got - ref) <= tol), (l, h)
+
+
+# Bar of the e4m3 path against the UNQUANTISED fp64 oracle, per head, fixed from
+# the format before any GPU comparison: e4m3 keeps 3 mantissa bits, so every
+# rounding of Q, K, V and P moves an element by at most u = 2^-4 of itself; the
+# output may sit on average half a unit roundoff, and at its worst element one
+# unit roundoff, away from the exact attention, relative to the output's own
+# scale (mean |O| and max |O| of the head).
+FP8_MEAN_REL, FP8_MAX_REL = 2.0 ** -5, 2.0 ** -4
+
+
+def test_step_fp8_480p_against_the_unquantised_oracle(cuda_device):
+    """The whole e4m3 step at 480P, every query row of every head, against the
+    exact fp64 attention over the unquantised kept cache (the kept lists are the
+    GPU's, which the bf16 parity tests check against the oracle's selection)."""
+    w = wl.get("480p")
+    x = wl.generate(w)
+    p = fkv.params_for(w)
+    d = parity.upload(x)
+    o = fkv.allocate(p)
+    c = fkv.allocate_fp8(p)
+    fkv.step_fp8(p, d, o, c)
+    assert fkv.read_status(o["ws"])[0] == 0
+    got_all = o["out"].cpu()
+    worst = (0.0, 0.0)
+    for h in range(w.H):
+        kept = parity.gpu_kept({"kept_cnt": o["kept_cnt"].cpu(), "kept_idx": o["kept_idx"].cpu()}, 0, h)
+        f64 = lambda k: wl.as_float64(x[k][0, h])  # noqa: E731
+        keys = np.concatenate([orc.compact(f64("k_hist"), kept, w.T), f64("k_cur")])
+        vals = np.concatenate([orc.compact(f64("v_hist"), kept, w.T), f64("v_cur")])
+        ref = orc.attention(f64("q_cur"), keys, vals, w.scale)
+        err = np.abs(got_all[0, h].double().numpy() - ref)
+        mean_rel = err.mean() / np.abs(ref).mean()
+        max_rel = err.max() / np.abs(ref).max()
+        worst = (max(worst[0], mean_rel), max(worst[1], max_rel))
+        assert mean_rel <= FP8_MEAN_REL and max_rel <= FP8_MAX_REL, (h, mean_rel, max_rel)
+    print("e4m3 vs unquantised oracle (mean/mean|O|, max/max|O|):", worst)

@@ -156,3 +156,33 @@ def test_tolerance_covers_simulated_evaluation(lag):
     # and the bound is not vacuous: a dropped V scale breaks it
     wrong = _simulated_fp8_attention(q, k, vc, np.ones_like(sv_key), 0.125, lag) * sv_key.max()
     assert np.any(np.abs(wrong - ref) > tol)
+
+
+def test_quantisation_alone_is_inside_the_stated_e4m3_bar():
+    """The bar the e4m3 GPU path is held to against the unquantised oracle
+    (mean-abs <= 2^-5 mean|O|, max-abs <= 2^-4 max|O| per head) must already
+    hold for the exact attention over the oracle's dequantised cache, with
+    room left for the kernel's own e4m3 rounding of the probabilities: here
+    at most half the bar, on one 480P head, every query row."""
+    import fkv_workloads as wl
+    from oracle import fkv_oracle as orc
+    w = wl.scaled(wl.get("480p"), name="fp8_bar", H=2, n_static=1, seed=5)
+    x = wl.generate(w)
+    f32 = lambda t: wl.as_float64(t).astype(np.float32)  # noqa: E731
+    h, kept = 1, np.array([0, 1, 3, 4, 6, 7, 9, 10, 12, 13, 15, 16, 17])
+    T = w.T
+    kc, sk, vc, sv = f8.compact_quantized(f32(x["k_hist"][0, h]), f32(x["v_hist"][0, h]), kept, T)
+    kq, skq = f8.quantize_segments(f32(x["k_cur"][0, h]), T)
+    vq, svq = f8.quantize_segments(f32(x["v_cur"][0, h]), T)
+    qq, sqq = f8.quantize_rows(f32(x["q_cur"][0, h]))
+    q8 = f8.e4m3_decode(qq) * sqq.astype(np.float64)[:, None]
+    k8 = np.concatenate([f8.dequantize(kc, sk, T), f8.dequantize(kq, skq, T)])
+    v8 = np.concatenate([f8.dequantize(vc, sv, T), f8.dequantize(vq, svq, T)])
+    f64 = lambda k: wl.as_float64(x[k][0, h])  # noqa: E731
+    keys = np.concatenate([orc.compact(f64("k_hist"), kept, T), f64("k_cur")])
+    vals = np.concatenate([orc.compact(f64("v_hist"), kept, T), f64("v_cur")])
+    exact = orc.attention(f64("q_cur"), keys, vals, w.scale)
+    quant = orc.attention(q8, k8, v8, w.scale)
+    err = np.abs(quant - exact)
+    assert err.mean() / np.abs(exact).mean() <= 0.5 * 2.0 ** -5
+    assert err.max() / np.abs(exact).max() <= 0.5 * 2.0 ** -4

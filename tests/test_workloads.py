@@ -50,3 +50,10 @@ def test_token_workload_budget():
 def test_sample_rows_covers_ends():
     r = wl.sample_rows(4680, 64, 3)
     assert r[0] == 0 and r[-1] == 4679 and len(np.unique(r)) == len(r)
+
+
+def test_tile_rows_hit_every_tile_and_both_ends():
+    for n in (4680, 24480, 128, 129, 37):
+        r = wl.tile_rows(n, seed=5)
+        assert r[0] == 0 and r[-1] == n - 1 and np.all(np.diff(r) > 0)
+        assert set(range(-(-n // 128))) <= set((r // 128).tolist())

@@ -66,7 +66,7 @@ def test_noalloc_matches_workspace_scoring_twice(cuda_device, case):
 def test_noalloc_rejects_scratch_above_its_maximum(cuda_device):
     w = wl.get("480p_30layer")  # 30 layers of per-block partial statistics: about 200 MB
     p = fkv.params_for(w)
-    assert fkv.sizes(p)["ws_bytes"] > 4 << 20
+    assert fkv.sizes(p)["ws_bytes"] > 16 << 20  # above the static maximum
     sentinel = torch.full((w.L, w.H, w.F), 7.0, device="cuda")
     dummy = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
     st = _noalloc(p, {"q_cur": dummy, "k_hist": dummy,

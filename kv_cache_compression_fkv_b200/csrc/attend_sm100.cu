@@ -57,6 +57,11 @@
 namespace fkv {
 namespace sm100 {
 
+// The MMA issuer tests the next group's K / V barrier inside the current
+// group's MMA issue (1) or waits on it in front of the next group (0).
+#ifndef FKV_ISSUE_LOOKAHEAD
+#define FKV_ISSUE_LOOKAHEAD 1
+#endif
 #ifndef FKV_ATTN_K_STAGES
 #define FKV_ATTN_K_STAGES 3
 #endif
@@ -250,6 +255,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       // softmax's bounded wait on it runs out (the MMAs themselves are issued
       // and complete; nothing else is left outstanding behind the signal).
       bool withhold = a.withhold_s0 != 0 && blockIdx.x == 0;
+      bool kf_ok = false, vf_ok = false;  // next K / V stage seen complete ahead of use
       const uint64_t dq = kmajor_desc(smem_u32(sm + kOffQ), 0);
       const uint64_t dk0 = kmajor_desc(smem_u32(sm + kOffK), 0);
       const uint64_t dv0 = mnmajor_desc(smem_u32(sm + kOffV), 0);
@@ -258,6 +264,43 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         const Unit t = decode(a, tile);
         bool o_free_seen = false;
         // O_h += P_h V for the stream's next block (`first`: its first of the unit).
+        // K and V stages are consumed in load order, so the K stage of the S
+        // group that follows a PV group, and the V stage of the PV group that
+        // follows an S group, are known in advance: each group tests that
+        // stage's barrier without blocking, inside its own MMA issue (kf_ok /
+        // vf_ok), and the next group waits only when the test saw it pending.
+#if FKV_ISSUE_LOOKAHEAD
+        auto issue_pv = [&](int h, bool first) -> bool {
+          if (!o_free_seen) {
+            if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort, a.wait_cycles)) return false;
+            o_free_seen = true;
+          }
+          if (!vf_ok && !mbar_wait(&bars->v_full[vs], vph, abort, a.wait_cycles)) return false;
+          if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort, a.wait_cycles)) return false;
+          ++p_use[h];
+          tc_fence_after();
+          // step k: P columns 8k.., V rows 16k.. (2048 B = 128 descriptor units)
+          kf_ok = mma8_ts_probe(tmem + col_o(h), tmem + col_s(h),
+                                dv0 + uint64_t(vs * kStageDesc), kIdescPV, first ? 0u : 1u,
+                                &bars->k_full[ks], kph) != 0;
+          vf_ok = false;
+          if (++vs == kVStages) { vs = 0; vph ^= 1; }
+          return true;
+        };
+        // S_h = Q K^T for the stream's next block.
+        auto issue_s = [&](int h) -> bool {
+          if (!kf_ok && !mbar_wait(&bars->k_full[ks], kph, abort, a.wait_cycles)) return false;
+          kf_ok = false;
+          // step k of the 128-deep contraction: 32 bytes along a 128-byte
+          // swizzled row, then the second 64-column region
+          vf_ok = mma8_ss_probe(tmem + col_s(h), dq, dk0 + uint64_t(ks * kStageDesc), kIdescQK,
+                                0u, &bars->v_full[vs], vph) != 0;
+          if (withhold && h == 0) withhold = false;
+          else mma_commit(&bars->s_full[h]);
+          if (++ks == kKStages) { ks = 0; kph ^= 1; }
+          return true;
+        };
+#else
         auto issue_pv = [&](int h, bool first) -> bool {
           if (!o_free_seen) {
             if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort, a.wait_cycles)) return false;
@@ -291,6 +334,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           if (++ks == kKStages) { ks = 0; kph ^= 1; }
           return true;
         };
+#endif
         if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort, a.wait_cycles))) break;
         // Order per step j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j) -- the load
         // order of K and of V.  Where stream 1 has one block fewer, its last

@@ -160,6 +160,80 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Eight kind::f16 MMAs into D (K = 8 x 16; the first accumulates only when
+// acc_first != 0) with a non-blocking test of an mbarrier phase placed before
+// them in the same instruction stream and read only after the eighth, so the
+// test's shared-memory round trip overlaps the MMA issue.  Returns 1 when the
+// phase of the given parity had completed at the time of the test.  The
+// operand addresses of step k are formed inside from the step-0 ones, so the
+// issuing thread keeps few registers live.
+//   mma8_ss_probe: A and B K-major in shared memory, both advancing as
+//                  kmajor_desc does (32 B per step, the next 64-element
+//                  region after step 3);
+//   mma8_ts_probe: A from tensor memory (8 columns per step), B MN-major in
+//                  shared memory (2048 B per step).
+__device__ __forceinline__ uint32_t mma8_ss_probe(uint32_t d, uint64_t a0, uint64_t b0,
+                                                  uint32_t idesc, uint32_t acc_first,
+                                                  uint64_t* bar, uint32_t parity) {
+  static_assert(kRegionBytes >> 4 == 1024, "descriptor step of the second region");
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred t, p, one;\n\t.reg .b64 a, b;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 t, [%5], %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 one, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], %2, %3, %7, p;\n\t"
+      "add.s64 a, %2, 2;\n\tadd.s64 b, %3, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 4;\n\tadd.s64 b, %3, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 6;\n\tadd.s64 b, %3, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 1024;\n\tadd.s64 b, %3, 1024;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 1026;\n\tadd.s64 b, %3, 1026;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 1028;\n\tadd.s64 b, %3, 1028;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 1030;\n\tadd.s64 b, %3, 1030;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], a, b, %7, one;\n\t"
+      "selp.u32 %0, 1, 0, t;\n\t}\n"
+      : "=r"(ok)
+      : "r"(d), "l"(a0), "l"(b0), "r"(acc_first), "r"(smem_u32(bar)), "r"(parity), "r"(idesc)
+      : "memory");
+  return ok;
+}
+__device__ __forceinline__ uint32_t mma8_ts_probe(uint32_t d, uint32_t a0, uint64_t b0,
+                                                  uint32_t idesc, uint32_t acc_first,
+                                                  uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred t, p, one;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 t, [%5], %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 one, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [%2], %3, %7, p;\n\t"
+      "add.u32 a, %2, 8;\n\tadd.s64 b, %3, 128;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 16;\n\tadd.s64 b, %3, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 24;\n\tadd.s64 b, %3, 384;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 32;\n\tadd.s64 b, %3, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 40;\n\tadd.s64 b, %3, 640;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 48;\n\tadd.s64 b, %3, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 56;\n\tadd.s64 b, %3, 896;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%1], [a], b, %7, one;\n\t"
+      "selp.u32 %0, 1, 0, t;\n\t}\n"
+      : "=r"(ok)
+      : "r"(d), "r"(a0), "l"(b0), "r"(acc_first), "r"(smem_u32(bar)), "r"(parity), "r"(idesc)
+      : "memory");
+  return ok;
+}
+
 // Arrives once on `bar` when every MMA issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(

@@ -203,7 +203,10 @@ int32_t fkv_workspace_init(void* ws, size_t bytes, void* stream);
  * Either output pointer may be NULL. */
 int32_t fkv_read_status(const void* ws, void* stream, int32_t* device_status, int32_t* detail);
 
-/* Step 2: segment scores.
+/* Step 2: segment scores.  Forcing-KV (ai-feeds.com/i/paper/2605.09681),
+ * "关键模块" 3: a dynamic head's history is grouped by frame and each group
+ * is scored by the current chunk's queries; Deep Forcing (bxzpzcl.cn/news/
+ * 2125000) section 3.1 step 2 for the token variant's phi_j.
  * Frame mode (dynamic heads only; static rows of seg_score are written 0):
  *   seg_score[l][h][f] = sum_i sum_{j in frame f} softmax_j(scale * q_i . k_j),
  *   q_i = q_cur[l][h][i*score_stride], softmax over the N history keys (and
@@ -247,7 +250,10 @@ int32_t fkv_score_segments_noalloc(const fkv_params_t* p, const void* q_cur, con
                                    const void* k_hist, const void* k_cur,
                                    const uint8_t* head_role, float* seg_score, void* stream);
 
-/* Steps 1 and 3: kept segment lists.
+/* Steps 1 and 3: kept segment lists.  Forcing-KV "关键模块" 2 (static heads:
+ * fixed positions taken out by mask) and 3 (dynamic heads: the most similar
+ * segments kept); Deep Forcing section 3.1 steps 1 and 3 (sink and recent
+ * regions kept, top C = N - S - R candidates).
  * Frame mode: static heads keep the frames with static_mask == 1; dynamic
  *   heads keep the k_per_head[l][h] frames of largest seg_score, ties to the
  *   lower frame.  kept_idx[l][h][0..cnt) ascending, kept_cnt[l][h] = cnt.
@@ -259,7 +265,8 @@ int32_t fkv_select_topk(const fkv_params_t* p, const float* seg_score, const uin
                         const uint8_t* static_mask, const int32_t* k_per_head, int32_t* kept_idx,
                         int32_t* kept_cnt, void* ws, void* stream);
 
-/* Step 4: compaction.  For each (l, h), copies the history rows of the kept
+/* Step 4: compaction.  Forcing-KV "输出与工程收益": the pruned KV tensors
+ * replace the original cache.  For each (l, h), copies the history rows of the kept
  * segments, in kept_idx order, into rows 0 .. kept_cnt*seg_len - 1 of
  * k_comp / v_comp (seg_len = T or 1).  Bit-exact copy.  Rows past that are
  * left untouched.  More rows than comp_rows: the copy is clamped and
@@ -268,7 +275,9 @@ int32_t fkv_compact_gather(const fkv_params_t* p, const void* k_hist, const void
                            const int32_t* kept_idx, const int32_t* kept_cnt, void* k_comp,
                            void* v_comp, void* ws, void* stream);
 
-/* Step 5: out[l][h][i] = sum_j softmax_j(scale * q_i . key_j) value_j with the
+/* Step 5.  Forcing-KV "输出与工程收益" (the compressed KV takes the original
+ * cache's place in the attention) and "与现有产品/工作流的接口" step 2.
+ * out[l][h][i] = sum_j softmax_j(scale * q_i . key_j) value_j with the
  * keys = k_comp rows 0 .. kept_cnt*seg_len - 1 followed by the Lq rows of
  * k_cur (no causal mask), values likewise.  float32 accumulation; the output
  * is rounded to the activation dtype.  Compressed rows past the kept count
@@ -317,8 +326,9 @@ int32_t fkv_cache_advance(const fkv_params_t* p, const void* k_comp, const void*
                           int64_t out_segments, void* k_next, void* v_next, void* ws,
                           void* stream);
 
-/* Steps 1-5 in one call: score (dynamic / token heads), select, compact,
- * attend, all enqueued on `stream` in that order. */
+/* Steps 1-5 in one call (Forcing-KV "方法": "输入与整体流程", "关键模块" 2-3,
+ * "输出与工程收益"): score (dynamic / token heads), select, compact, attend,
+ * all enqueued on `stream`, each step after the one it reads from. */
 int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void* stream);
 
 /* ---- Comparison selectors --------------------------------------------------

@@ -92,7 +92,7 @@ constexpr float kRescaleLog2 = 8.0f;
 static_assert(kProductionWaitCycles == kWaitCycles, "one production wait limit");
 // One of every FKV_POLY_EVERY exponential pairs goes to the FMA-pipe exp2 (0: none).
 #ifndef FKV_POLY_EVERY
-#define FKV_POLY_EVERY 0
+#define FKV_POLY_EVERY 8
 #endif
 
 __host__ __device__ constexpr uint32_t col_s(int h) { return 128u * uint32_t(h); }
@@ -179,6 +179,9 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // Everything above is on-chip; global memory (kept counts, Q/K/V, the
+  // output) is touched only once the kernel before this one has completed.
+  pdl_wait();
   if (warp >= 8) {
     regs_decrease<kControlRegs>();
   if (warp == kProducerWarp) {
@@ -584,8 +587,8 @@ cudaError_t launch_attend_sm100(const Dims& d, const void* q_cur, const void* k_
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(kAttnSmem));
   if (e != cudaSuccess) return e;
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();
-  attend_sm100_kernel<<<grid, kAttnThreads, kAttnSmem, s>>>(tq, tkc, tvc, tkn, tvn, a);
-  return cudaGetLastError();
+  return launch_kernel(attend_sm100_kernel, dim3(grid), dim3(kAttnThreads), kAttnSmem, s, d.pdl,
+                       tq, tkc, tvc, tkn, tvn, a);
 }
 
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s) {

@@ -440,13 +440,21 @@ int32_t fkv_step(const fkv_params_t* p, const fkv_step_io_t* io, void* ws, void*
   if ((st = do_score(d, io->q_cur, io->q_score, io->k_hist, io->k_cur, io->head_role,
                      io->seg_score, ws, s)))
     return st;
-  if ((st = do_select(d, io->seg_score, io->head_role, io->static_mask, io->k_per_head,
+  // Every kernel after the scoring follows one of this call's own kernels on
+  // the stream: launch it as a programmatic dependent (its on-chip prologue
+  // overlaps the previous kernel's tail; it waits for that grid before it
+  // touches global memory).  Without scoring work the select kernel is the
+  // first of the call and launches normally.
+  Dims dp = d;
+  dp.pdl = d.token ? d.nseg > 0 : d.F > 0;
+  if ((st = do_select(dp, io->seg_score, io->head_role, io->static_mask, io->k_per_head,
                       io->kept_idx, io->kept_cnt, ws, s)))
     return st;
-  if ((st = do_gather(d, io->k_hist, io->v_hist, io->kept_idx, io->kept_cnt, io->k_comp,
+  dp.pdl = true;
+  if ((st = do_gather(dp, io->k_hist, io->v_hist, io->kept_idx, io->kept_cnt, io->k_comp,
                       io->v_comp, ws, s)))
     return st;
-  return do_attend(d, io->q_cur, io->k_cur, io->v_cur, io->k_comp, io->v_comp, io->kept_cnt,
+  return do_attend(dp, io->q_cur, io->k_cur, io->v_cur, io->k_comp, io->v_comp, io->kept_cnt,
                    io->out, ws, s);
 }
 

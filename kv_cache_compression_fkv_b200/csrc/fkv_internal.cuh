@@ -29,6 +29,7 @@ struct Dims {
   bool score_with_chunk;  // frame mode: chunk keys in the scoring normaliser
   bool static_token_mask; // frame mode: per-token static masks, kept lists in tokens
   int elem;          // bytes per activation element
+  bool pdl = false;  // launch as a programmatic dependent of the previous kernel
 };
 
 // Layout of the frame-mode partial softmax statistics (part_ml, float2
@@ -68,6 +69,40 @@ struct WsLayout {
 };
 
 WsLayout ws_layout(const Dims& d);
+
+// Programmatic dependent launch.  Inside one call sequence (fkv_step), every
+// kernel after the first is launched so that the launch is prepared while its
+// predecessor on the stream is still running and its CTAs start as soon as
+// that grid has finished; it runs its on-chip prologue (shared-memory
+// barriers, tensor memory, tensor-map prefetch), then pdl_wait() blocks until
+// the predecessor grid has completed and its memory is visible -- before the
+// kernel reads or writes any global memory.  No kernel signals its
+// dependents early (griddepcontrol.launch_dependents): measured, dependents
+// resident while their predecessor still runs slowed it down more than the
+// early start saved.  Launched without the attribute, pdl_wait() returns at
+// once.
+#ifndef FKV_PDL
+#define FKV_PDL 1
+#endif
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launches `kernel`, as a programmatic dependent of the previous work on `s`
+// when `pdl` is set.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (pdl && FKV_PDL) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 // Records the first device-side error of a call sequence.
 __device__ __forceinline__ void report(int32_t* status, int32_t code, int32_t detail) {

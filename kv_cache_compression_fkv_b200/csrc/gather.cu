@@ -22,6 +22,7 @@ gather_kernel(int32_t seg_len, int32_t nseg_total, int32_t max_kept, int32_t com
               const uint4* __restrict__ v_hist, const int32_t* __restrict__ kept_idx,
               const int32_t* __restrict__ kept_cnt, uint4* __restrict__ k_comp,
               uint4* __restrict__ v_comp, int32_t* status) {
+  pdl_wait();
   const int lh = blockIdx.y;
   int32_t cnt = kept_cnt[lh];
   if (cnt < 0 || cnt > max_kept) {
@@ -83,12 +84,12 @@ cudaError_t launch_gather(const Dims& d, const void* k_hist, const void* v_hist,
   if (bx < 1) bx = 1;
   if (bx > 65535) bx = 65535;
   dim3 grid(unsigned(bx), unsigned(d.LH));
-  gather_kernel<<<grid, kGatherThreads, 0, s>>>(
-      int32_t(d.seg_len), int32_t(d.seg_len == 1 ? d.N : d.F), int32_t(d.max_kept),
-      int32_t(d.comp_rows), vec_per_row, d.N, static_cast<const uint4*>(k_hist),
-      static_cast<const uint4*>(v_hist), kept_idx, kept_cnt, static_cast<uint4*>(k_comp),
-      static_cast<uint4*>(v_comp), status);
-  return cudaGetLastError();
+  return launch_kernel(gather_kernel, grid, dim3(kGatherThreads), 0, s, d.pdl,
+                       int32_t(d.seg_len), int32_t(d.seg_len == 1 ? d.N : d.F),
+                       int32_t(d.max_kept), int32_t(d.comp_rows), vec_per_row, d.N,
+                       static_cast<const uint4*>(k_hist), static_cast<const uint4*>(v_hist),
+                       kept_idx, kept_cnt, static_cast<uint4*>(k_comp),
+                       static_cast<uint4*>(v_comp), status);
 }
 
 // Next history cache: rows [0, keep*seg_len) of the output are the last

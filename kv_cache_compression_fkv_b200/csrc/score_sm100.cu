@@ -36,6 +36,12 @@ namespace sm100 {
 #ifndef FKV_SCORE_CTAS_PER_SM
 #define FKV_SCORE_CTAS_PER_SM 2
 #endif
+#ifndef FKV_SCORE_POLY_EVERY
+#define FKV_SCORE_POLY_EVERY 0
+#endif
+constexpr int kScorePolyEvery = FKV_SCORE_POLY_EVERY;
+constexpr int kScorePolyDiv = kScorePolyEvery > 0 ? kScorePolyEvery : 1;
+static_assert(FKV_POLY_DEG == 3, "scores need the degree-3 exp2 (8.6e-5)");
 constexpr int kScoreStages = FKV_SCORE_STAGES;
 constexpr int kScoreCtasPerSm = FKV_SCORE_CTAS_PER_SM;
 constexpr int kScoreThreads = 320;
@@ -334,7 +340,10 @@ score_sm100_kernel(const __grid_constant__ CUtensorMap tm_qs,
       for (int i = 0; i < 32; ++i) {
         const float2 e = ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])),
                                sl2x2, negm2);
-        acc[i & 3] = fadd2(acc[i & 3], make_float2(ex2(e.x), ex2(e.y)));
+        // one pair in FKV_SCORE_POLY_EVERY on the FMA pipe (relative error
+        // <= 8.6e-5 per term), the rest on MUFU
+        const bool poly = kScorePolyEvery > 0 && i % kScorePolyDiv == kScorePolyDiv - 1;
+        acc[i & 3] = fadd2(acc[i & 3], poly ? exp2_poly2(e) : make_float2(ex2(e.x), ex2(e.y)));
       }
       const float2 s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
       const float2 mine = make_float2(m, m == -INFINITY ? 0.f : s2.x + s2.y);

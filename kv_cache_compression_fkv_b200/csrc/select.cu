@@ -25,6 +25,7 @@ __global__ void select_frame_kernel(int F, const float* __restrict__ seg_score,
                                     int32_t* __restrict__ kept_cnt, int32_t* status) {
   extern __shared__ uint32_t keys[];
   __shared__ int warp_counts[32];
+  pdl_wait();
   const int lh = blockIdx.x;
   const int f = threadIdx.x;
   const bool dyn = head_role ? head_role[lh] != 0 : true;  // no roles: every head ranked
@@ -74,9 +75,9 @@ cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uin
                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                 cudaStream_t s) {
   const int threads = d.F <= 32 ? 32 : ((d.F + 31) / 32) * 32;
-  select_frame_kernel<<<d.LH, threads, sizeof(uint32_t) * (d.F > 0 ? d.F : 1), s>>>(
-      d.F, seg_score, head_role, static_mask, k_per_head, kept_idx, kept_cnt, status);
-  return cudaGetLastError();
+  return launch_kernel(select_frame_kernel, dim3(d.LH), dim3(threads),
+                       sizeof(uint32_t) * (d.F > 0 ? d.F : 1), s, d.pdl, d.F, seg_score, head_role,
+                       static_mask, k_per_head, kept_idx, kept_cnt, status);
 }
 
 // ---------------------------------------------------------------------------
@@ -98,6 +99,7 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
   __shared__ int warp_tot[kSelWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int64_t s_need;
+  pdl_wait();
   const int lh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const float* ph = phi + int64_t(lh) * n_c;
@@ -218,6 +220,7 @@ select_frame_tokens_kernel(int F, int T, int64_t N, const float* __restrict__ se
   __shared__ int32_t kf[1024];
   __shared__ int warp_tot[kSelWarps];
   __shared__ int s_cnt;
+  pdl_wait();
   const int lh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int32_t* out = kept_idx + int64_t(lh) * N;
@@ -285,10 +288,9 @@ cudaError_t launch_select_frame_tokens(const Dims& d, const float* seg_score,
                                        const uint8_t* head_role, const uint8_t* static_mask,
                                        const int32_t* k_per_head, int32_t* kept_idx,
                                        int32_t* kept_cnt, int32_t* status, cudaStream_t s) {
-  select_frame_tokens_kernel<<<d.LH, kSelThreads, 0, s>>>(d.F, d.T, d.N, seg_score, head_role,
-                                                          static_mask, k_per_head, kept_idx,
-                                                          kept_cnt, status);
-  return cudaGetLastError();
+  return launch_kernel(select_frame_tokens_kernel, dim3(d.LH), dim3(kSelThreads), 0, s, d.pdl,
+                       d.F, d.T, d.N, seg_score, head_role, static_mask, k_per_head, kept_idx,
+                       kept_cnt, status);
 }
 
 cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int32_t* k_per_head,
@@ -300,9 +302,9 @@ cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(sizeof(uint32_t) * kSelCacheKeys));
   if (e != cudaSuccess) return e;
-  select_token_kernel<<<d.LH, kSelThreads, smem, s>>>(d.nseg, d.S, d.R, d.N, cached, seg_score,
-                                                      k_per_head, kept_idx, kept_cnt, status);
-  return cudaGetLastError();
+  return launch_kernel(select_token_kernel, dim3(d.LH), dim3(kSelThreads), smem, s, d.pdl,
+                       d.nseg, d.S, d.R, d.N, cached, seg_score, k_per_head, kept_idx, kept_cnt,
+                       status);
 }
 
 }  // namespace fkv

@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kRowWarps * 32)
 score_rows_kernel(int F, int split, int chunk, int E, int64_t n_s,
                   const uint8_t* __restrict__ head_role, float2* __restrict__ part_ml,
                   float2* __restrict__ row_ml) {
+  pdl_wait();
   const int lh = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t i = int64_t(blockIdx.x) * kRowWarps + warp;
@@ -184,6 +185,7 @@ score_frames_kernel(int F, int split, int E, int64_t n_s, const uint8_t* __restr
                     const float2* __restrict__ part_ml, float* __restrict__ seg_score,
                     const int32_t* __restrict__ poison) {
   __shared__ float wsum[kFrameThreads / 32];
+  pdl_wait();
   const int f = blockIdx.x, lh = blockIdx.y;
   float* out = seg_score + int64_t(lh) * F + f;
   if (!head_role[lh]) {
@@ -234,15 +236,15 @@ cudaError_t launch_score_frame_finalize(const Dims& d, const ScoreLayout& sl,
                                         const int32_t* poison) {
   if (d.n_s > 0) {
     dim3 grid(unsigned((d.n_s + kRowWarps - 1) / kRowWarps), unsigned(d.LH));
-    score_rows_kernel<<<grid, kRowWarps * 32, 0, s>>>(d.F, sl.split, sl.chunk, sl.E, d.n_s,
-                                                      head_role, part_ml, row_ml);
-    cudaError_t e = cudaGetLastError();
+    // both finalize kernels follow this call's statistics kernel on the stream
+    cudaError_t e = launch_kernel(score_rows_kernel, grid, dim3(kRowWarps * 32), 0, s, true, d.F,
+                                  sl.split, sl.chunk, sl.E, d.n_s, head_role, part_ml, row_ml);
     if (e != cudaSuccess) return e;
   }
   if (d.F < 1) return cudaSuccess;
-  score_frames_kernel<<<dim3(unsigned(d.F), unsigned(d.LH)), kFrameThreads, 0, s>>>(
-      d.F, sl.split, sl.E, d.n_s, head_role, part_ml, seg_score, poison);
-  return cudaGetLastError();
+  return launch_kernel(score_frames_kernel, dim3(unsigned(d.F), unsigned(d.LH)),
+                       dim3(kFrameThreads), 0, s, true, d.F, sl.split, sl.E, d.n_s, head_role,
+                       static_cast<const float2*>(part_ml), seg_score, poison);
 }
 
 // ---------------------------------------------------------------------------

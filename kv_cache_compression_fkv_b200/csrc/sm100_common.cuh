@@ -368,18 +368,28 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
 // adding 1.5*2^23 rounded toward -inf, which leaves it in the low mantissa
 // bits; shifting those bits by 23 yields n << 23 modulo 2^32.  x is clamped
 // to >= -127 so that -inf gives exactly +0.  Valid for x <= 127.
+#ifndef FKV_POLY_DEG
+#define FKV_POLY_DEG 3
+#endif
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {
   const float kMagic = 12582912.0f;  // 1.5 * 2^23
-  const float c1 = __uint_as_float(0x3f31f335u);  // 6.951172948e-01
-  const float c2 = __uint_as_float(0x3e691b63u);  // 2.276435345e-01
-  const float c3 = __uint_as_float(0x3d9dd5d8u);  // 7.706803083e-02
   x.x = fmaxf(x.x, -127.f);
   x.y = fmaxf(x.y, -127.f);
   const float2 mg = make_float2(kMagic, kMagic);
   const float2 y = fadd2_rm(x, mg);
   const float2 f = fsub2(x, fsub2(y, mg));
+#if FKV_POLY_DEG == 2
+  // degree-2 fit: max relative error 2.05e-3 on [0, 1]
+  const float c1 = __uint_as_float(0x3f2a7c6au);  // 6.659609079e-01
+  const float c2 = __uint_as_float(0x3ea8ece9u);  // 3.299324811e-01
+  float2 p = ffma2(make_float2(c2, c2), f, make_float2(c1, c1));
+#else
+  const float c1 = __uint_as_float(0x3f31f335u);  // 6.951172948e-01
+  const float c2 = __uint_as_float(0x3e691b63u);  // 2.276435345e-01
+  const float c3 = __uint_as_float(0x3d9dd5d8u);  // 7.706803083e-02
   float2 p = ffma2(make_float2(c3, c3), f, make_float2(c2, c2));
   p = ffma2(p, f, make_float2(c1, c1));
+#endif
   p = ffma2(p, f, make_float2(1.f, 1.f));
   return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
                      __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));

@@ -74,6 +74,7 @@ constexpr int kPhiUnroll = 4;  // row pairs in flight per warp
 __global__ void __launch_bounds__(kPhiThreads)
 phi_bf16_kernel(int64_t N, int64_t S, int64_t n_c, const uint4* __restrict__ k_hist,
                 const float* __restrict__ qbar, float* __restrict__ phi) {
+  pdl_wait();
   const int lh = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane & 15;      // 16-byte chunk of the row: dims 8*sub .. 8*sub+7
@@ -154,8 +155,11 @@ cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k
     if (per_head > need) per_head = need;
     if (per_head < 1) per_head = 1;
     dim3 grid(unsigned(per_head), unsigned(d.LH));
-    phi_bf16_kernel<<<grid, kPhiThreads, 0, s>>>(d.N, d.S, d.nseg,
-                                                 static_cast<const uint4*>(k_hist), qbar, seg_score);
+    // follows this call's q-sum kernel on the stream
+    cudaError_t e = launch_kernel(phi_bf16_kernel, grid, dim3(kPhiThreads), 0, s, true, d.N, d.S,
+                                  d.nseg, static_cast<const uint4*>(k_hist),
+                                  static_cast<const float*>(qbar), seg_score);
+    if (e != cudaSuccess) return e;
   } else {
     const int warps = 8;
     int64_t bx = (d.nseg + warps - 1) / warps;

@@ -12,8 +12,9 @@ from pinned host memory and the output read back inside the timed region.
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events
 on the launching stream; between timed steps the L2 is flushed by writing a
 256 MiB buffer outside the events.  The per-kernel breakdown (roofline) comes
-from a second timed pass that calls the four entry points one by one with
-events between them.  N > 1: one process per GPU (torchrun), each rank runs
+from a second timed pass over the four entry points, each captured into a
+CUDA graph and replayed between events (so that a short kernel's time is not
+inflated by the Python binding's host work in front of it).  N > 1: one process per GPU (torchrun), each rank runs
 its own independent chunk step (replicas: the step has no exchange), and the
 time is the max over ranks.
 
@@ -205,6 +206,53 @@ def aggregate_throughput(units_per_rank, world, max_ms):
     return units_per_rank * world / (max_ms / 1e3)
 
 
+def graphed(fn):
+    """fn (one or more library calls on the current stream) captured into a
+    CUDA graph: a replay runs exactly fn's kernels with no host work between
+    them, so an event pair around it times the GPU alone (the Python binding's
+    argument checks would otherwise leave the GPU idle in front of a short
+    kernel).  The library allocates nothing and never synchronises, so its calls
+    capture as they are."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graphs(graphs, flush, steps, stream):
+    """Mean device time of each graph of `graphs` (replayed in order), with the
+    L2 flushed before each round."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
+          for _ in range(steps)]
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        ev[i][0].record(stream)
+        for k, g in enumerate(graphs):
+            g.replay()
+            ev[i][k + 1].record(stream)
+    torch.cuda.synchronize()
+    return [statistics.mean(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps))
+            for k in range(len(graphs))]
+
+
+def entry_point_calls(fkv, p, x, outs):
+    """The four entry points of the step as separate calls, in step order."""
+    return [
+        lambda: fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"],
+                                   x.get("head_role"), outs["seg_score"], outs["ws"],
+                                   k_cur=x["k_cur"]),
+        lambda: fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
+                                x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"]),
+        lambda: fkv.compact_gather(p, x["k_hist"], x["v_hist"], outs["kept_idx"],
+                                   outs["kept_cnt"], outs["k_comp"], outs["v_comp"], outs["ws"]),
+        lambda: fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"],
+                                      outs["v_comp"], outs["kept_cnt"], outs["out"], outs["ws"]),
+    ]
+
+
 def kept_per_head(w):
     """Segments every head keeps in the workload's step: the static mask size
     (= the dynamic budget k) in frame mode, S + C + R tokens in token mode."""
@@ -257,29 +305,13 @@ def measure_workload(fkv, w, x_cpu, dev, steps, warmup, flush):
         evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     step_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
-    for i in range(steps):
-        flush.fill_(i & 0xFF)
-        e = kev[i]
-        e[0].record(stream)
-        fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
-                           outs["seg_score"], outs["ws"], k_cur=x["k_cur"])
-        e[1].record(stream)
-        fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
-                        x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])
-        e[2].record(stream)
-        fkv.compact_gather(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
-                           outs["k_comp"], outs["v_comp"], outs["ws"])
-        e[3].record(stream)
-        fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"],
-                              outs["v_comp"], outs["kept_cnt"], outs["out"], outs["ws"])
-        e[4].record(stream)
-    torch.cuda.synchronize(dev)
+    graphs = [graphed(f) for f in entry_point_calls(fkv, p, x, outs)]
     st, det = fkv.read_status(outs["ws"])
     if st != 0:
         raise RuntimeError(f"device status {st} on head {det} ({w.name})")
-    part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(steps))
-            for j, n in enumerate(["score", "select", "gather", "attend"])}
+    part = dict(zip(["score", "select", "gather", "attend"],
+                    time_graphs(graphs, flush, steps, stream)))
+    del graphs
     alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
                       else torch.ones(w.L, w.H))
     peaks, _ = load_peaks()
@@ -337,19 +369,18 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # warm-up
-    for _ in range(args.warmup):
-        fkv.step(p, x, outs, io=io)
-    torch.cuda.synchronize(dev)
-    st, det = fkv.read_status(outs["ws"])
-    if st != 0:
-        raise RuntimeError(f"device status {st} on head {det}")
-
-    # ---- timed: fused fkv_step, inputs resident
+    # ---- timed: fused fkv_step, inputs resident.  The clock sampler starts
+    # before the warm-up, so the GPU is not left idle between warm-up and timing.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
-    barrier()
     with ClockSampler(local_rank) as clk:
+        for _ in range(args.warmup):
+            fkv.step(p, x, outs, io=io)
+        torch.cuda.synchronize(dev)
+        st, det = fkv.read_status(outs["ws"])
+        if st != 0:
+            raise RuntimeError(f"device status {st} on head {det}")
+        barrier()
         for i in range(args.steps):
             flush.fill_(i & 0xFF)
             evs[i][0].record(stream)
@@ -365,46 +396,26 @@ def run_ours(args, rank, world, local_rank):
     rope = w.granularity == "frame" and not w.static_token_mask
     # temporal RoPE band of the re-positioning compaction: 22 pairs (44 dims)
     omega = (10000.0 ** (-torch.arange(22, dtype=torch.float32) / 22)).to(dev)
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    calls = entry_point_calls(fkv, p, x, outs)
+    if rope:
+        calls.append(lambda: fkv.compact_gather_rope(p, x["k_hist"], x["v_hist"], outs["kept_idx"],
+                                                     outs["kept_cnt"], omega, outs["k_comp"],
+                                                     outs["v_comp"], outs["ws"]))
     barrier()
-    for i in range(args.steps):
-        flush.fill_(i & 0xFF)
-        e = kev[i]
-        e[0].record(stream)
-        fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
-                           outs["seg_score"], outs["ws"], k_cur=x["k_cur"])
-        e[1].record(stream)
-        fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
-                        x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])
-        e[2].record(stream)
-        fkv.compact_gather(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
-                           outs["k_comp"], outs["v_comp"], outs["ws"])
-        e[3].record(stream)
-        fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"], outs["v_comp"],
-                              outs["kept_cnt"], outs["out"], outs["ws"])
-        e[4].record(stream)
-        if rope:
-            fkv.compact_gather_rope(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
-                                    omega, outs["k_comp"], outs["v_comp"], outs["ws"])
-        e[5].record(stream)
-    torch.cuda.synchronize(dev)
+    graphs = [graphed(f) for f in calls]
+    times = time_graphs(graphs, flush, args.steps, stream)
+    del graphs
     barrier()
-    part = {n: statistics.mean(kev[i][j].elapsed_time(kev[i][j + 1]) for i in range(args.steps))
-            for j, n in enumerate(["score", "select", "gather", "attend", "gather_rope"])}
+    part = dict(zip(["score", "select", "gather", "attend", "gather_rope"], times + [0.0]))
 
     # comparison selectors (uniform eviction / random drop), same budgets
-    hev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        hev[i][0].record(stream)
-        fkv.select_heuristic(p, "uniform", 1, x["k_per_head"], outs["kept_idx"], outs["kept_cnt"],
-                             outs["ws"])
-        hev[i][1].record(stream)
-        fkv.select_heuristic(p, "random", 1 + i, x["k_per_head"], outs["kept_idx"], outs["kept_cnt"],
-                             outs["ws"], seg_score=outs["seg_score"])
-        hev[i][2].record(stream)
-    torch.cuda.synchronize(dev)
-    heur = {n: statistics.mean(hev[i][j].elapsed_time(hev[i][j + 1]) for i in range(args.steps))
-            for j, n in enumerate(["uniform", "random"])}
+    hg = [graphed(lambda: fkv.select_heuristic(p, "uniform", 1, x["k_per_head"], outs["kept_idx"],
+                                                 outs["kept_cnt"], outs["ws"])),
+          graphed(lambda: fkv.select_heuristic(p, "random", 1, x["k_per_head"], outs["kept_idx"],
+                                                 outs["kept_cnt"], outs["ws"],
+                                                 seg_score=outs["seg_score"]))]
+    heur = dict(zip(["uniform", "random"], time_graphs(hg, flush, args.steps, stream)))
+    del hg
 
     # ---- FP8 (e4m3) compressed cache: the same scoring and selection, then the
     # e4m3 compaction, the chunk's quantisation and the kind::f8f6f4 attention
@@ -413,31 +424,20 @@ def run_ours(args, rank, world, local_rank):
             and w.T >= 128):
         c8 = fkv.allocate_fp8(p, dev)
         out8 = torch.empty_like(outs["out"])
-        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
-        for i in range(args.warmup + args.steps):
-            flush.fill_(i & 0xFF)
-            e = fev[i - args.warmup] if i >= args.warmup else None
-            if e: e[0].record(stream)  # noqa: E701
-            fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"], x.get("head_role"),
-                               outs["seg_score"], outs["ws"], k_cur=x["k_cur"])
-            if e: e[1].record(stream)  # noqa: E701
-            fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
-                            x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"])
-            if e: e[2].record(stream)  # noqa: E701
-            fkv.compact_gather_fp8(p, x["k_hist"], x["v_hist"], outs["kept_idx"], outs["kept_cnt"],
-                                   c8, outs["ws"])
-            if e: e[3].record(stream)  # noqa: E701
-            fkv.quantize_chunk_fp8(p, x["q_cur"], x["k_cur"], x["v_cur"], c8, outs["ws"])
-            if e: e[4].record(stream)  # noqa: E701
-            fkv.attend_compressed_fp8(p, c8, outs["kept_cnt"], out8, outs["ws"])
-            if e: e[5].record(stream)  # noqa: E701
-        torch.cuda.synchronize(dev)
+        calls8 = entry_point_calls(fkv, p, x, outs)[:2] + [
+            lambda: fkv.compact_gather_fp8(p, x["k_hist"], x["v_hist"], outs["kept_idx"],
+                                           outs["kept_cnt"], c8, outs["ws"]),
+            lambda: fkv.quantize_chunk_fp8(p, x["q_cur"], x["k_cur"], x["v_cur"], c8, outs["ws"]),
+            lambda: fkv.attend_compressed_fp8(p, c8, outs["kept_cnt"], out8, outs["ws"]),
+        ]
+        g8 = [graphed(f) for f in calls8]
         st, det = fkv.read_status(outs["ws"])
         if st != 0:
             raise RuntimeError(f"device status {st} on head {det} (fp8 path)")
-        fp8 = {n: statistics.mean(fev[i][j].elapsed_time(fev[i][j + 1]) for i in range(args.steps))
-               for j, n in enumerate(["score", "select", "gather", "quant", "attend"])}
-        fp8["step"] = statistics.mean(fev[i][0].elapsed_time(fev[i][5]) for i in range(args.steps))
+        fp8 = dict(zip(["score", "select", "gather", "quant", "attend"],
+                       time_graphs(g8, flush, args.steps, stream)))
+        del g8
+        fp8["step"] = sum(fp8[n] for n in ("score", "select", "gather", "quant", "attend"))
         # the same step through the one fused call (fkv_step_fp8)
         sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]

@@ -122,6 +122,59 @@ __device__ __forceinline__ void mma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The issuer's lookahead form of the four MMAs of a group (see mma8_ss_probe):
+// a non-blocking test of the next group's K / V barrier is issued before the
+// MMAs and read after them.  Step k: A and B 32 bytes (2 descriptor units)
+// further along the row (S), or A 8 tensor-memory columns and B 32 keys = 4 KB
+// (256 descriptor units) further (P.V).
+__device__ __forceinline__ uint32_t mma4_ss_e4m3_probe(uint32_t d, uint64_t a0, uint64_t b0,
+                                                       uint32_t idesc, uint32_t acc_first,
+                                                       uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred t, p, one;\n\t.reg .b64 a, b;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 t, [%5], %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 one, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], %2, %3, %7, p;\n\t"
+      "add.s64 a, %2, 2;\n\tadd.s64 b, %3, 2;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 4;\n\tadd.s64 b, %3, 4;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %7, one;\n\t"
+      "add.s64 a, %2, 6;\n\tadd.s64 b, %3, 6;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %7, one;\n\t"
+      "selp.u32 %0, 1, 0, t;\n\t}\n"
+      : "=r"(ok)
+      : "r"(d), "l"(a0), "l"(b0), "r"(acc_first), "r"(smem_u32(bar)), "r"(parity), "r"(idesc)
+      : "memory");
+  return ok;
+}
+__device__ __forceinline__ uint32_t mma4_ts_e4m3_probe(uint32_t d, uint32_t a0, uint64_t b0,
+                                                       uint32_t idesc, uint32_t acc_first,
+                                                       uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred t, p, one;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 t, [%5], %6;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 one, 0, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [%2], %3, %7, p;\n\t"
+      "add.u32 a, %2, 8;\n\tadd.s64 b, %3, 256;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 16;\n\tadd.s64 b, %3, 512;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %7, one;\n\t"
+      "add.u32 a, %2, 24;\n\tadd.s64 b, %3, 768;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %7, one;\n\t"
+      "selp.u32 %0, 1, 0, t;\n\t}\n"
+      : "=r"(ok)
+      : "r"(d), "r"(a0), "l"(b0), "r"(acc_first), "r"(smem_u32(bar)), "r"(parity), "r"(idesc)
+      : "memory");
+  return ok;
+}
+#ifndef FKV_F8_ISSUE_LOOKAHEAD
+#define FKV_F8_ISSUE_LOOKAHEAD 0
+#endif
+
 // K-major e4m3 tile: rows 128 B apart, 8-row groups 1024 B apart; step k
 // (32 elements) lives 32 B further along the row.
 __device__ __forceinline__ uint64_t kmajor8_desc(uint32_t tile_saddr, int k) {
@@ -239,6 +292,7 @@ attend_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       uint32_t uc = 0, ks = 0, kph = 0, vs = 0, vph = 0;
       uint32_t p_use[2] = {0, 0};
       bool ok = true;
+      bool kf_ok = false, vf_ok = false;  // next K / V stage seen complete ahead of use
       const uint64_t dq = kmajor8_desc(smem_u32(sm + kOffQ), 0);
       const uint64_t dk0 = kmajor8_desc(smem_u32(sm + kOffK), 0);
       const uint64_t dv0 = mnmajor8_desc(smem_u32(sm + kOffV), 0);
@@ -252,27 +306,42 @@ attend_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort)) return false;
             o_free_seen = true;
           }
-          if (!mbar_wait(&bars->v_full[vs], vph, abort)) return false;
+          if (!vf_ok && !mbar_wait(&bars->v_full[vs], vph, abort)) return false;
           if (!mbar_wait(&bars->p_full[h], p_use[h] & 1, abort)) return false;
           ++p_use[h];
           tc_fence_after();
           // step k: 32 keys = 4 KB further (descriptor address field: bytes >> 4)
           const uint64_t dv = dv0 + uint64_t(vs * kStageDesc);
+#if FKV_F8_ISSUE_LOOKAHEAD
+          // K and V stages are consumed in load order: test the K stage of the
+          // S group that comes next while these MMAs issue
+          kf_ok = mma4_ts_e4m3_probe(tmem + col_o(h), tmem + col_s(h), dv, kIdescPV,
+                                     first ? 0u : 1u, &bars->k_full[ks], kph) != 0;
+#else
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_ts_e4m3(tmem + col_o(h), tmem + col_s(h) + k * 8, dv + uint64_t(k) * 256u,
                         kIdescPV, (first && k == 0) ? 0u : 1u);
+#endif
+          vf_ok = false;
           if (++vs == kStages) { vs = 0; vph ^= 1; }
           return true;
         };
         // S_h = Q K^T for the stream's next block; step k: 32 bytes along the row.
         auto issue_s = [&](int h) -> bool {
-          if (!mbar_wait(&bars->k_full[ks], kph, abort)) return false;
+          if (!kf_ok && !mbar_wait(&bars->k_full[ks], kph, abort)) return false;
+          kf_ok = false;
           const uint64_t dk = dk0 + uint64_t(ks * kStageDesc);
+#if FKV_F8_ISSUE_LOOKAHEAD
+          // ... and the V stage of the P.V group that comes next
+          vf_ok = mma4_ss_e4m3_probe(tmem + col_s(h), dq, dk, kIdescQK, 0u, &bars->v_full[vs],
+                                     vph) != 0;
+#else
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_ss_e4m3(tmem + col_s(h), dq + uint64_t(2 * k), dk + uint64_t(2 * k), kIdescQK,
                         k > 0 ? 1u : 0u);
+#endif
           mma_commit(&bars->s_full[h]);
           if (++ks == kStages) { ks = 0; kph ^= 1; }
           return true;

@@ -96,6 +96,7 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
                     int32_t* status) {
   extern __shared__ uint32_t skeys[];
   __shared__ unsigned hist[256];
+  __shared__ unsigned whist[kSelWarps][256];  // one histogram per warp
   __shared__ int warp_tot[kSelWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int64_t s_need;
@@ -119,15 +120,18 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
   }
   auto key_at = [&](int64_t j) -> uint32_t { return cached ? skeys[j] : ordered_key(ph[j]); };
 
-  // Radix select of the C-th largest key, most significant byte first.  Lanes
-  // of a warp that hit the same bin are merged (__match_any_sync) into one
-  // shared-memory atomic, so clustered scores do not serialise the histogram.
+  // Radix select of the C-th largest key, most significant byte first.  Each
+  // warp counts into a histogram of its own (lanes that hit the same bin are
+  // merged by __match_any_sync into one shared-memory add), so the many keys
+  // that share a bin -- scores of one magnitude share their top byte -- never
+  // contend across warps; the 32 histograms are then summed per bin in warp
+  // order.
   uint32_t prefix = 0, pmask = 0;
   int64_t need = C;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int b = tid; b < 256; b += kSelThreads) hist[b] = 0;
-    __syncthreads();
+    for (int b = lane; b < 256; b += 32) whist[warp][b] = 0;
+    __syncwarp();
     for (int64_t base = int64_t(warp) * 32; base < n_c; base += kSelThreads) {
       const int64_t j = base + lane;
       uint32_t bin = 256;  // no bin
@@ -136,7 +140,15 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
         if ((key & pmask) == prefix) bin = (key >> shift) & 255u;
       }
       const unsigned grp = __match_any_sync(0xffffffffu, bin);
-      if (bin < 256 && lane == __ffs(grp) - 1) atomicAdd(&hist[bin], unsigned(__popc(grp)));
+      if (bin < 256 && lane == __ffs(grp) - 1) whist[warp][bin] += unsigned(__popc(grp));
+      __syncwarp();
+    }
+    __syncthreads();
+    if (tid < 256) {
+      unsigned c = 0;
+#pragma unroll 8
+      for (int w = 0; w < kSelWarps; ++w) c += whist[w][tid];
+      hist[tid] = c;
     }
     __syncthreads();
     if (warp == 0) {

@@ -40,6 +40,7 @@ qsum_kernel(int D, int64_t n_q, const T* __restrict__ q_score, float* __restrict
 // 16-byte load per row; 64 row groups (r = g mod 64) summed in order, then
 // the 64 group sums per dim added in a fixed order.
 constexpr int kQsumRowGroups = 64;
+constexpr int kQsumBatch = 8;
 __global__ void __launch_bounds__(1024)
 qsum_bf16_kernel(int64_t n_q, const uint4* __restrict__ q_score, float* __restrict__ qbar) {
   __shared__ float part[kQsumRowGroups][128];
@@ -47,14 +48,25 @@ qsum_bf16_kernel(int64_t n_q, const uint4* __restrict__ q_score, float* __restri
   const int sub = threadIdx.x & 15, g = threadIdx.x >> 4;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   const uint4* q = q_score + int64_t(lh) * n_q * 16 + sub;
-  for (int64_t r = g; r < n_q; r += kQsumRowGroups) {
-    const uint4 v = __ldcs(q + r * 16);
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  // kQsumBatch rows of the group loaded before any is added (bytes in flight),
+  // then added in row order
+  for (int64_t r0 = g; r0 < n_q; r0 += int64_t(kQsumBatch) * kQsumRowGroups) {
+    uint4 v[kQsumBatch];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
-      acc[2 * e] += __low2float(b);
-      acc[2 * e + 1] += __high2float(b);
+    for (int u = 0; u < kQsumBatch; ++u) {
+      const int64_t r = r0 + int64_t(u) * kQsumRowGroups;
+      v[u] = r < n_q ? __ldcs(q + r * 16) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < kQsumBatch; ++u) {
+      if (r0 + int64_t(u) * kQsumRowGroups >= n_q) break;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w[e]);
+        acc[2 * e] += __low2float(b);
+        acc[2 * e + 1] += __high2float(b);
+      }
     }
   }
 #pragma unroll

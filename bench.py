@@ -12,9 +12,10 @@ from pinned host memory and the output read back inside the timed region.
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events
 on the launching stream; between timed steps the L2 is flushed by writing a
 256 MiB buffer outside the events.  The per-kernel breakdown (roofline) comes
-from a second timed pass over the four entry points, each captured into a
-CUDA graph and replayed between events (so that a short kernel's time is not
-inflated by the Python binding's host work in front of it).  N > 1: one process per GPU (torchrun), each rank runs
+from a second timed pass over the four entry points, each a C-ABI call whose
+arguments were checked and converted once (``fkv.marshal``), with events
+between them (so that a short kernel's time is not inflated by the Python
+binding's host work in front of it).  N > 1: one process per GPU (torchrun), each rank runs
 its own independent chunk step (replicas: the step has no exchange), and the
 time is the max over ranks.
 
@@ -206,50 +207,38 @@ def aggregate_throughput(units_per_rank, world, max_ms):
     return units_per_rank * world / (max_ms / 1e3)
 
 
-def graphed(fn):
-    """fn (one or more library calls on the current stream) captured into a
-    CUDA graph: a replay runs exactly fn's kernels with no host work between
-    them, so an event pair around it times the GPU alone (the Python binding's
-    argument checks would otherwise leave the GPU idle in front of a short
-    kernel).  The library allocates nothing and never synchronises, so its calls
-    capture as they are."""
-    fn()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        fn()
-    torch.cuda.synchronize()
-    return g
-
-
-def time_graphs(graphs, flush, steps, stream):
-    """Mean device time of each graph of `graphs` (replayed in order), with the
-    L2 flushed before each round."""
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)]
+def time_calls(calls, flush, steps, stream):
+    """Mean device time of each call of `calls` (pairs (c_function, c_args)
+    from ``fkv.marshal``, issued in order), with the L2 flushed before each
+    round.  The calls carry no Python-side work, so the GPU never waits on the
+    host in front of a short kernel."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
           for _ in range(steps)]
     for i in range(steps):
         flush.fill_(i & 0xFF)
         ev[i][0].record(stream)
-        for k, g in enumerate(graphs):
-            g.replay()
+        for k, (fn, args) in enumerate(calls):
+            st = fn(*args)
+            if st != 0:
+                raise RuntimeError(f"{fn.__name__}: status {st}")
             ev[i][k + 1].record(stream)
     torch.cuda.synchronize()
     return [statistics.mean(ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps))
-            for k in range(len(graphs))]
+            for k in range(len(calls))]
 
 
 def entry_point_calls(fkv, p, x, outs):
-    """The four entry points of the step as separate calls, in step order."""
+    """The four entry points of the step as separate C-ABI calls, in step order."""
     return [
-        lambda: fkv.score_segments(p, x["q_cur"], x.get("q_score"), x["k_hist"],
-                                   x.get("head_role"), outs["seg_score"], outs["ws"],
-                                   k_cur=x["k_cur"]),
-        lambda: fkv.select_topk(p, outs["seg_score"], x.get("head_role"), x.get("static_mask"),
-                                x["k_per_head"], outs["kept_idx"], outs["kept_cnt"], outs["ws"]),
-        lambda: fkv.compact_gather(p, x["k_hist"], x["v_hist"], outs["kept_idx"],
-                                   outs["kept_cnt"], outs["k_comp"], outs["v_comp"], outs["ws"]),
-        lambda: fkv.attend_compressed(p, x["q_cur"], x["k_cur"], x["v_cur"], outs["k_comp"],
-                                      outs["v_comp"], outs["kept_cnt"], outs["out"], outs["ws"]),
+        fkv.marshal(fkv.score_segments, p, x["q_cur"], x.get("q_score"), x["k_hist"],
+                    x.get("head_role"), outs["seg_score"], outs["ws"], k_cur=x["k_cur"]),
+        fkv.marshal(fkv.select_topk, p, outs["seg_score"], x.get("head_role"),
+                    x.get("static_mask"), x["k_per_head"], outs["kept_idx"], outs["kept_cnt"],
+                    outs["ws"]),
+        fkv.marshal(fkv.compact_gather, p, x["k_hist"], x["v_hist"], outs["kept_idx"],
+                    outs["kept_cnt"], outs["k_comp"], outs["v_comp"], outs["ws"]),
+        fkv.marshal(fkv.attend_compressed, p, x["q_cur"], x["k_cur"], x["v_cur"],
+                    outs["k_comp"], outs["v_comp"], outs["kept_cnt"], outs["out"], outs["ws"]),
     ]
 
 
@@ -305,13 +294,11 @@ def measure_workload(fkv, w, x_cpu, dev, steps, warmup, flush):
         evs[i][1].record(stream)
     torch.cuda.synchronize(dev)
     step_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    graphs = [graphed(f) for f in entry_point_calls(fkv, p, x, outs)]
+    part = dict(zip(["score", "select", "gather", "attend"],
+                    time_calls(entry_point_calls(fkv, p, x, outs), flush, steps, stream)))
     st, det = fkv.read_status(outs["ws"])
     if st != 0:
         raise RuntimeError(f"device status {st} on head {det} ({w.name})")
-    part = dict(zip(["score", "select", "gather", "attend"],
-                    time_graphs(graphs, flush, steps, stream)))
-    del graphs
     alg = algorithmic(w, outs["kept_cnt"].cpu(), x_cpu["head_role"] if w.granularity == "frame"
                       else torch.ones(w.L, w.H))
     peaks, _ = load_peaks()
@@ -398,24 +385,20 @@ def run_ours(args, rank, world, local_rank):
     omega = (10000.0 ** (-torch.arange(22, dtype=torch.float32) / 22)).to(dev)
     calls = entry_point_calls(fkv, p, x, outs)
     if rope:
-        calls.append(lambda: fkv.compact_gather_rope(p, x["k_hist"], x["v_hist"], outs["kept_idx"],
-                                                     outs["kept_cnt"], omega, outs["k_comp"],
-                                                     outs["v_comp"], outs["ws"]))
+        calls.append(fkv.marshal(fkv.compact_gather_rope, p, x["k_hist"], x["v_hist"],
+                                 outs["kept_idx"], outs["kept_cnt"], omega, outs["k_comp"],
+                                 outs["v_comp"], outs["ws"]))
     barrier()
-    graphs = [graphed(f) for f in calls]
-    times = time_graphs(graphs, flush, args.steps, stream)
-    del graphs
+    times = time_calls(calls, flush, args.steps, stream)
     barrier()
     part = dict(zip(["score", "select", "gather", "attend", "gather_rope"], times + [0.0]))
 
     # comparison selectors (uniform eviction / random drop), same budgets
-    hg = [graphed(lambda: fkv.select_heuristic(p, "uniform", 1, x["k_per_head"], outs["kept_idx"],
-                                                 outs["kept_cnt"], outs["ws"])),
-          graphed(lambda: fkv.select_heuristic(p, "random", 1, x["k_per_head"], outs["kept_idx"],
-                                                 outs["kept_cnt"], outs["ws"],
-                                                 seg_score=outs["seg_score"]))]
-    heur = dict(zip(["uniform", "random"], time_graphs(hg, flush, args.steps, stream)))
-    del hg
+    hc = [fkv.marshal(fkv.select_heuristic, p, "uniform", 1, x["k_per_head"], outs["kept_idx"],
+                      outs["kept_cnt"], outs["ws"]),
+          fkv.marshal(fkv.select_heuristic, p, "random", 1, x["k_per_head"], outs["kept_idx"],
+                      outs["kept_cnt"], outs["ws"], seg_score=outs["seg_score"])]
+    heur = dict(zip(["uniform", "random"], time_calls(hc, flush, args.steps, stream)))
 
     # ---- FP8 (e4m3) compressed cache: the same scoring and selection, then the
     # e4m3 compaction, the chunk's quantisation and the kind::f8f6f4 attention
@@ -425,18 +408,18 @@ def run_ours(args, rank, world, local_rank):
         c8 = fkv.allocate_fp8(p, dev)
         out8 = torch.empty_like(outs["out"])
         calls8 = entry_point_calls(fkv, p, x, outs)[:2] + [
-            lambda: fkv.compact_gather_fp8(p, x["k_hist"], x["v_hist"], outs["kept_idx"],
-                                           outs["kept_cnt"], c8, outs["ws"]),
-            lambda: fkv.quantize_chunk_fp8(p, x["q_cur"], x["k_cur"], x["v_cur"], c8, outs["ws"]),
-            lambda: fkv.attend_compressed_fp8(p, c8, outs["kept_cnt"], out8, outs["ws"]),
+            fkv.marshal(fkv.compact_gather_fp8, p, x["k_hist"], x["v_hist"], outs["kept_idx"],
+                        outs["kept_cnt"], c8, outs["ws"]),
+            fkv.marshal(fkv.quantize_chunk_fp8, p, x["q_cur"], x["k_cur"], x["v_cur"], c8,
+                        outs["ws"]),
+            fkv.marshal(fkv.attend_compressed_fp8, p, c8, outs["kept_cnt"], out8, outs["ws"]),
         ]
-        g8 = [graphed(f) for f in calls8]
+        time_calls(calls8, flush, args.warmup, stream)  # warm-up
+        fp8 = dict(zip(["score", "select", "gather", "quant", "attend"],
+                       time_calls(calls8, flush, args.steps, stream)))
         st, det = fkv.read_status(outs["ws"])
         if st != 0:
             raise RuntimeError(f"device status {st} on head {det} (fp8 path)")
-        fp8 = dict(zip(["score", "select", "gather", "quant", "attend"],
-                       time_graphs(g8, flush, args.steps, stream)))
-        del g8
         fp8["step"] = sum(fp8[n] for n in ("score", "select", "gather", "quant", "attend"))
         # the same step through the one fused call (fkv_step_fp8)
         sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))

@@ -30,7 +30,7 @@ __all__ = [
     "FkvError", "Params", "make_params", "params_for", "sizes", "allocate", "score_segments",
     "select_topk", "compact_gather", "attend_compressed", "step", "read_status", "library",
     "step_launches", "make_step_io", "score_segments_noalloc", "cache_advance",
-    "compact_gather_rope",
+    "compact_gather_rope", "marshal",
 ]
 
 
@@ -198,7 +198,7 @@ def score_segments(p: Params, q_cur, q_score, k_hist, head_role, seg_score, ws, 
 def score_segments_noalloc(p: Params, q_cur, q_score, k_hist, head_role, seg_score, stream=None,
                            k_cur=None):
     """score_segments without a workspace: for callers that cannot allocate
-    device memory.  The library's own static 4 MiB device scratch is used, so
+    device memory.  The library's own static 16 MiB device scratch is used, so
     sizes needing more are rejected, and calls must not overlap on the GPU."""
     n, dt = _shapes(p), _act_dtype(p)
     token = p.granularity == _lib.FKV_GRAN_TOKEN
@@ -425,6 +425,43 @@ def step_fp8(p: Params, inputs: Dict[str, torch.Tensor], outputs: Dict[str, torc
     st = _lib.load().fkv_step_fp8(ctypes.byref(p), ctypes.byref(io), ctypes.byref(fp),
                                   outputs["ws"].data_ptr(), _stream(stream))
     _check(st, "fkv_step_fp8")
+
+
+class _Recorder:
+    """Stands in for the loaded library while one wrapper runs: records the C
+    function and its converted arguments instead of calling it."""
+
+    def __init__(self, lib):
+        self._lib = lib
+        self.call = None
+
+    def __getattr__(self, name):
+        fn = getattr(self._lib, name)
+
+        def record(*args):
+            self.call = (fn, args)
+            return _lib.FKV_OK
+        return record
+
+
+def marshal(wrapper, *args, **kwargs):
+    """(c_function, c_args) of one call of an entry-point wrapper of this
+    module, checked and converted once: ``c_function(*c_args)`` repeats the
+    call with no Python-side work (for timing loops, or a serving loop that
+    calls the same entry point on the same buffers; the status it returns is
+    the caller's to check).  Nothing is launched by marshal itself.  The
+    recorded arguments refer to the given tensors and params, which must
+    stay alive."""
+    real = _lib.load
+    rec = _Recorder(real())
+    _lib.load = lambda: rec
+    try:
+        wrapper(*args, **kwargs)
+    finally:
+        _lib.load = real
+    if rec.call is None:
+        raise ValueError(f"{getattr(wrapper, '__name__', wrapper)} made no library call")
+    return rec.call
 
 
 def read_status(ws: torch.Tensor, stream=None):

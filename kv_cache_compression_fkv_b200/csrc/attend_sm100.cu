@@ -62,12 +62,6 @@ namespace sm100 {
 #ifndef FKV_ISSUE_LOOKAHEAD
 #define FKV_ISSUE_LOOKAHEAD 1
 #endif
-// P handed over by one arrival per softmax warp after a warp barrier (1), or
-// one arrival per softmax thread (0).
-#ifndef FKV_WARP_ARRIVE
-#define FKV_WARP_ARRIVE 0
-#endif
-constexpr uint32_t kPArrivals = FKV_WARP_ARRIVE ? 4u : 128u;
 #ifndef FKV_ATTN_K_STAGES
 #define FKV_ATTN_K_STAGES 3
 #endif
@@ -168,7 +162,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     for (int h = 0; h < 2; ++h) {
       mbar_init(&bars->s_full[h], 1);
-      mbar_init(&bars->p_full[h], kPArrivals);
+      mbar_init(&bars->p_full[h], 128);
     }
     mbar_init(&bars->o_ready, 1);
     mbar_init(&bars->o_free, kSoftmaxThreads);
@@ -479,12 +473,7 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
           fence_proxy_async_smem();
         }
         tc_fence_before();
-#if FKV_WARP_ARRIVE
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->p_full[h]);
-#else
         mbar_arrive(&bars->p_full[h]);
-#endif
       }
       if (!ok) break;
       // V stage of this stream's last PV (released once both PV chains are done)

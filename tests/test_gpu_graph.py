@@ -53,3 +53,30 @@ def test_step_graph_replay_matches_eager(cuda_device, name):
             for h in range(w.H):
                 c = int(cnt[l, h])
                 assert torch.equal(gi[l, h, :c], ri[l, h, :c]), (l, h)
+
+
+def test_marshalled_calls_repeat_the_wrapper_calls(cuda_device):
+    """fkv.marshal: one wrapper call checked and converted once, repeated as a
+    bare C-ABI call, gives the same results as the wrapper."""
+    w = wl.scaled(wl.get("480p"), name="marshal", H=4, T=256, F=6, Fc=2, n_static=2,
+                  static_frames=(0, 2, 5), k_dynamic=3, score_stride=4, seed=33)
+    x = parity.upload(wl.generate(w))
+    p = fkv.params_for(w)
+    ref, o = fkv.allocate(p), fkv.allocate(p)
+    fkv.step(p, x, ref)
+    calls = [
+        fkv.marshal(fkv.score_segments, p, x["q_cur"], None, x["k_hist"], x["head_role"],
+                    o["seg_score"], o["ws"]),
+        fkv.marshal(fkv.select_topk, p, o["seg_score"], x["head_role"], x["static_mask"],
+                    x["k_per_head"], o["kept_idx"], o["kept_cnt"], o["ws"]),
+        fkv.marshal(fkv.compact_gather, p, x["k_hist"], x["v_hist"], o["kept_idx"],
+                    o["kept_cnt"], o["k_comp"], o["v_comp"], o["ws"]),
+        fkv.marshal(fkv.attend_compressed, p, x["q_cur"], x["k_cur"], x["v_cur"], o["k_comp"],
+                    o["v_comp"], o["kept_cnt"], o["out"], o["ws"]),
+    ]
+    for _ in range(2):
+        for fn, args in calls:
+            assert fn(*args) == 0
+    assert fkv.read_status(o["ws"])[0] == 0
+    for k in ("seg_score", "kept_cnt", "out"):
+        assert torch.equal(o[k], ref[k]), k

@@ -84,6 +84,7 @@ cudaError_t launch_select_frame(const Dims& d, const float* seg_score, const uin
 
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kSelBatch = 8;  // key loads in flight per thread
 
 // Keys cached in shared memory when they fit (the 14B workload's 18720
 // candidates take 73 KB); otherwise every pass re-reads them (from L2).
@@ -98,6 +99,7 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
   __shared__ unsigned hist[256];
   __shared__ unsigned whist[kSelWarps][256];  // one histogram per warp
   __shared__ int warp_tot[kSelWarps];
+  __shared__ int warp_pre[kSelWarps + 1];
   __shared__ uint32_t s_prefix;
   __shared__ int64_t s_need;
   pdl_wait();
@@ -115,7 +117,20 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
   if (tid == 0) kept_cnt[lh] = int32_t(S + C + R);
   if (C == 0) return;
   if (cached) {
-    for (int64_t j = tid; j < n_c; j += kSelThreads) skeys[j] = ordered_key(ph[j]);
+    // kSelBatch independent loads in flight per thread before any is stored
+    for (int64_t j0 = tid; j0 < n_c; j0 += int64_t(kSelThreads) * kSelBatch) {
+      float v[kSelBatch];
+#pragma unroll
+      for (int u = 0; u < kSelBatch; ++u) {
+        const int64_t j = j0 + int64_t(u) * kSelThreads;
+        v[u] = j < n_c ? __ldcs(ph + j) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kSelBatch; ++u) {
+        const int64_t j = j0 + int64_t(u) * kSelThreads;
+        if (j < n_c) skeys[j] = ordered_key(v[u]);
+      }
+    }
     __syncthreads();
   }
   auto key_at = [&](int64_t j) -> uint32_t { return cached ? skeys[j] : ordered_key(ph[j]); };
@@ -199,13 +214,19 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
     const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
     if (lane == 0) warp_tot[warp] = int(__popc(bg) | (__popc(be) << 16));
     __syncthreads();
-    int before = 0, total = 0;
-    for (int w = 0; w < kSelWarps; ++w) {
-      const int c = warp_tot[w];
-      before += (w < warp) ? c : 0;
-      total += c;
+    if (warp == 0) {  // exclusive prefix of the packed (gt, eq) counts over the warps
+      const int c = warp_tot[lane];
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      warp_pre[lane] = incl - c;
+      if (lane == 31) warp_pre[32] = incl;
     }
     __syncthreads();
+    const int before = warp_pre[warp], total = warp_pre[32];
     const unsigned below = (1u << lane) - 1u;
     const int64_t gt_before = gt_seen + (before & 0xFFFF) + __popc(bg & below);
     const int64_t eq_before = eq_seen + (before >> 16) + __popc(be & below);

@@ -227,6 +227,36 @@ def time_calls(calls, flush, steps, stream):
             for k in range(len(calls))]
 
 
+def hw_rates(dev):
+    """The library's hardware-rate diagnostics (SM cycles, CTA 0 of one CTA
+    per SM): tcgen05.mma of the attention's shapes issued back to back by one
+    thread (Q.K^T and P.V through the attention's own grouped issue), and ex2
+    per warp with 1, 2 and 4 warps per sub-partition."""
+    from kv_cache_compression_fkv_b200 import _lib
+    lib = _lib.load()
+    cyc = torch.zeros(4, dtype=torch.int64, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    s = torch.cuda.current_stream(dev).cuda_stream
+    n = 256
+    mma = {}
+    for name, shape, busy in (("qk_ss_m128n128k16", 6, 0), ("pv_ts_m128n128k16", 7, 0),
+                              ("ss_m128n256k16", 2, 0), ("ss_m128n64k16", 3, 0),
+                              ("qk_with_two_busy_warps", 6, 1)):
+        for _ in range(2):
+            if lib.fkv_diag_mma_rate(shape, n, busy, cyc.data_ptr(), ws.data_ptr(), s) != 0:
+                return None
+        torch.cuda.synchronize(dev)
+        mma[name] = round(int(cyc[1]) / n, 1)
+    ex2 = {}
+    for warps in (1, 2, 4):
+        for _ in range(2):
+            if lib.fkv_diag_ex2_rate(4096, warps, cyc.data_ptr(), s) != 0:
+                return None
+        torch.cuda.synchronize(dev)
+        ex2[f"{warps}_warps_per_subpartition"] = round(int(cyc[0]) / 4096, 2)
+    return {"mma_cycles_per_instruction": mma, "ex2_cycles_per_warp_instruction": ex2}
+
+
 def entry_point_calls(fkv, p, x, outs):
     """The four entry points of the step as separate C-ABI calls, in step order."""
     return [
@@ -653,6 +683,8 @@ def run_ours(args, rank, world, local_rank):
                 line["workloads"][name] = measure_workload(
                     fkv, we, wl.generate(we), dev, min(args.steps, 10), args.warmup, flush)
         line["workloads_clocks"] = clk_x.summary()
+    if world == 1:
+        line["hw_rates"] = hw_rates(dev)
     if rank == 0 and not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(w, x_cpu, budget_s=args.cpu_budget)
     if dist is not None:

@@ -55,7 +55,7 @@ extern "C" {
 
 /* 3: adds fkv_fp8_cache_t and the three *_fp8 entry points;
  * 4: adds fkv_select_heuristic; 5: adds fkv_step_fp8;
- * 6: adds fkv_diag_attend_timeout. */
+ * 6: adds fkv_diag_attend_timeout, fkv_diag_mma_rate, fkv_diag_ex2_rate. */
 #define FKV_ABI_VERSION 6
 
 typedef enum fkv_status {
@@ -192,6 +192,29 @@ int32_t fkv_diag_attend_timeout(const fkv_params_t* p, const void* q_cur, const 
                                 const void* v_cur, const void* k_comp, const void* v_comp,
                                 const int32_t* kept_cnt, void* out, int64_t wait_cycles, void* ws,
                                 void* stream);
+
+/* Diagnostics of the hardware rates the attention kernel's design rests on
+ * (one CTA per SM; CTA 0 reports; no caller data is touched):
+ *  - fkv_diag_mma_rate: one thread issues n_mma (8..4096) tcgen05.mma
+ *    back to back into one accumulator, bf16 operands, fp32 accumulation;
+ *    shape 0 = M128 N128 K16 from shared memory, B K-major (the Q.K^T
+ *    step), 1 = M128 N128 K16 with A from tensor memory and an MN-major B
+ *    (the P.V step: V stored [keys][dims]), 2 = M128 N256, 3 = M128 N64,
+ *    4 = shape 0 with an MN-major B, 5 = shape 1 with a K-major B, 6 and 7
+ *    = shapes 0 and 1 issued eight at a time through the attention kernel's
+ *    own issue code; n_mma a multiple of 8.  busy != 0
+ *    keeps two more warps of the issuer's sub-partition
+ *    running an FMA + ex2 loop meanwhile.  cycles: device int64[4];
+ *    cycles[0] = SM cycles to issue the n MMAs, cycles[1] = until they have
+ *    completed.  ws: a workspace (>= 256 B, 256-B aligned) whose status word
+ *    records FKV_ERR_TIMEOUT if the completion wait gave up.
+ *  - fkv_diag_ex2_rate: `warps` (1..4) warps per SM sub-partition each run
+ *    n (multiple of 8, <= 2^20) ex2.approx.ftz.f32 in 8 independent chains;
+ *    cycles: device int64[2]; cycles[0] = SM cycles of one warp.
+ * Sizes out of range: FKV_ERR_SHAPE. */
+int32_t fkv_diag_mma_rate(int32_t shape, int32_t n_mma, int32_t busy, int64_t* cycles, void* ws,
+                          void* stream);
+int32_t fkv_diag_ex2_rate(int32_t n, int32_t warps, int64_t* cycles, void* stream);
 
 /* Zeroes the workspace (status word included) on `stream`.  Call once after
  * allocating it; entry points never clear the status word themselves. */

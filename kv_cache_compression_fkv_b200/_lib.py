@@ -77,6 +77,8 @@ SIGNATURES = {
     "fkv_exp2_emulated": (c_i32, [c_vp, c_vp, c_i64, c_vp]),
     "fkv_diag_attend_timeout": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp,
                                         c_vp, c_i64, c_vp, c_vp]),
+    "fkv_diag_mma_rate": (c_i32, [c_i32, c_i32, c_i32, c_vp, c_vp, c_vp]),
+    "fkv_diag_ex2_rate": (c_i32, [c_i32, c_i32, c_vp, c_vp]),
     "fkv_workspace_init": (c_i32, [c_vp, c_sz, c_vp]),
     "fkv_read_status": (c_i32, [c_vp, c_vp, ctypes.POINTER(c_i32), ctypes.POINTER(c_i32)]),
     "fkv_score_segments": (c_i32, [ctypes.POINTER(Params), c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),

@@ -259,6 +259,24 @@ int32_t fkv_exp2_emulated(const float* x, float* y, int64_t n, void* stream) {
   return cuda_status(launch_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream)));
 }
 
+int32_t fkv_diag_mma_rate(int32_t shape, int32_t n_mma, int32_t busy, int64_t* cycles, void* ws,
+                          void* stream) {
+  if (shape < 0 || shape > 7 || n_mma < 8 || n_mma > 4096 || n_mma % 8 != 0)
+    return FKV_ERR_SHAPE;
+  if (!cycles) return FKV_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FKV_ERR_WORKSPACE;
+  return cuda_status(launch_diag_mma_rate(shape, n_mma, busy != 0 ? 1 : 0,
+                                          reinterpret_cast<long long*>(cycles), status_ptr(ws),
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int32_t fkv_diag_ex2_rate(int32_t n, int32_t warps, int64_t* cycles, void* stream) {
+  if (n < 8 || n > (1 << 20) || n % 8 != 0 || warps < 1 || warps > 4) return FKV_ERR_SHAPE;
+  if (!cycles) return FKV_ERR_INVALID_ARG;
+  return cuda_status(launch_diag_ex2_rate(n, warps, reinterpret_cast<long long*>(cycles),
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int32_t fkv_workspace_init(void* ws, size_t bytes, void* stream) {
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || bytes < 256) return FKV_ERR_WORKSPACE;
   return cuda_status(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));

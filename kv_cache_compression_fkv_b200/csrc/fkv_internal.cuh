@@ -179,6 +179,11 @@ cudaError_t launch_advance(const Dims& d, int64_t out_segments, const void* k_co
                            const void* v_cur, void* k_next, void* v_next, int32_t* status,
                            cudaStream_t s);
 cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s);
+// Hardware-rate diagnostics (diag.cu): cycles of n tcgen05.mma of one shape
+// issued back to back by one thread, and of n ex2 per warp.
+cudaError_t launch_diag_mma_rate(int shape, int n, int busy, long long* cycles, int32_t* status,
+                                 cudaStream_t s);
+cudaError_t launch_diag_ex2_rate(int n, int warps, long long* cycles, cudaStream_t s);
 cudaError_t launch_quant_segments(const Dims& d, int n_slots, int64_t src_rows, int64_t dst_rows,
                                   const int32_t* kept_idx, const int32_t* kept_cnt,
                                   const void* src_k, const void* src_v, void* dst_k, void* dst_v,

@@ -10,8 +10,10 @@ layer).  ``value`` is whole-job throughput with the inputs resident in HBM;
 from pinned host memory and the output read back inside the timed region.
 
 Timing: W untimed warm-up steps, then K steps each bracketed by CUDA events
-on the launching stream; between timed steps the L2 is flushed by writing a
-256 MiB buffer outside the events.  The per-kernel breakdown (roofline) comes
+on the launching stream; between timed steps the L2 is flushed outside the
+events by writing a 256 MiB buffer and reading it back (the read evicts the
+written lines, so the timed kernels start on a cold L2 with no dirty lines of
+the flush left to write back).  The per-kernel breakdown (roofline) comes
 from a second timed pass over the four entry points, each a C-ABI call whose
 arguments were checked and converted once (``fkv.marshal``), with events
 between them (so that a short kernel's time is not inflated by the Python
@@ -207,6 +209,21 @@ def aggregate_throughput(units_per_rank, world, max_ms):
     return units_per_rank * world / (max_ms / 1e3)
 
 
+class L2Flush:
+    """Empties the L2 between timed steps: a 256 MiB write (twice the L2),
+    then a read of the same buffer, on the current stream, outside the
+    events.  After the read the L2 holds clean lines of the flush buffer, so a
+    timed kernel's misses do not also write back the flush's dirty lines."""
+
+    def __init__(self, dev):
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.sink = torch.empty(1, dtype=torch.int64, device=dev)
+
+    def __call__(self, i):
+        self.buf.fill_(i & 0xFF)
+        self.sink.copy_(self.buf.view(torch.int64).sum().view(1))
+
+
 def time_calls(calls, flush, steps, stream):
     """Mean device time of each call of `calls` (pairs (c_function, c_args)
     from ``fkv.marshal``, issued in order), with the L2 flushed before each
@@ -215,7 +232,7 @@ def time_calls(calls, flush, steps, stream):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
           for _ in range(steps)]
     for i in range(steps):
-        flush.fill_(i & 0xFF)
+        flush(i)
         ev[i][0].record(stream)
         for k, (fn, args) in enumerate(calls):
             st = fn(*args)
@@ -284,7 +301,7 @@ def bench_config(base, w, world=1, split="replicas", extra=None):
     """The ``config`` object of the JSON line; both arms print the same one."""
     cfg = {"workload": base.name, "L": base.L, "H": base.H, "D": w.D, "T": w.T, "F": w.F,
            "Fc": w.Fc, "granularity": w.granularity, "kept_per_head": kept_per_head(base),
-           "l2": "flushed between timed steps (256 MiB write outside the events)",
+           "l2": "flushed between timed steps (256 MiB written, then read, outside the events)",
            "parallelism": (f"heads split over {world} GPUs" if split == "heads" and world > 1
                            else f"replicas x{world}" if world > 1 else "single GPU")}
     cfg.update(extra or {})
@@ -318,7 +335,7 @@ def measure_workload(fkv, w, x_cpu, dev, steps, warmup, flush):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
     for i in range(steps):
-        flush.fill_(i & 0xFF)
+        flush(i)
         evs[i][0].record(stream)
         fkv.step(p, x, outs, io=io)
         evs[i][1].record(stream)
@@ -383,7 +400,7 @@ def run_ours(args, rank, world, local_rank):
     x = {k: v.to(dev) for k, v in x_cpu.items()}
     outs = fkv.allocate(p, dev)
     io = fkv.make_step_io(p, x, outs)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     def barrier():
         if dist is not None:
@@ -403,7 +420,7 @@ def run_ours(args, rank, world, local_rank):
             raise RuntimeError(f"device status {st} on head {det}")
         barrier()
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             evs[i][0].record(stream)
             fkv.step(p, x, outs, io=io)
             evs[i][1].record(stream)
@@ -459,7 +476,7 @@ def run_ours(args, rank, world, local_rank):
         sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(args.steps)]
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+            flush(i)
             sev[i][0].record(stream)
             fkv.step_fp8(p, x, outs, c8, io=io)
             sev[i][1].record(stream)
@@ -545,7 +562,7 @@ def run_ours(args, rank, world, local_rank):
             evs_ = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     for _ in range(args.steps)]
             for i in range(args.steps):
-                flush.fill_(i & 0xFF)
+                flush(i)
                 evs_[i][0].record(stream)
                 body()
                 evs_[i][1].record(stream)

@@ -89,19 +89,25 @@ constexpr int kSelBatch = 8;  // key loads in flight per thread
 // Keys cached in shared memory when they fit (the 14B workload's 18720
 // candidates take 73 KB); otherwise every pass re-reads them (from L2).
 constexpr int64_t kSelCacheKeys = 40960;
+// With at most kSelCandMaxKeys cached keys, the keys that survive the first
+// pass (those in the threshold's top-byte bin) are also copied to a list of
+// up to kSelCandKeys entries, and the later passes scan only that list.
+constexpr int64_t kSelCandMaxKeys = 24576;
+constexpr int64_t kSelCandKeys = 16384;
 
 __global__ void __launch_bounds__(kSelThreads)
-select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
+select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached, int cand_cap,
                     const float* __restrict__ phi, const int32_t* __restrict__ k_per_head,
                     int32_t* __restrict__ kept_idx, int32_t* __restrict__ kept_cnt,
                     int32_t* status) {
-  extern __shared__ uint32_t skeys[];
+  extern __shared__ uint32_t skeys[];  // [n_c] keys if cached, then [cand_cap] candidates
+  uint32_t* cand = skeys + (cached ? n_c : 0);
   __shared__ unsigned hist[256];
   __shared__ unsigned whist[kSelWarps][256];  // one histogram per warp
-  __shared__ int warp_tot[kSelWarps];
-  __shared__ int warp_pre[kSelWarps + 1];
+  __shared__ int warp_gt[kSelWarps], warp_eq[kSelWarps];
   __shared__ uint32_t s_prefix;
   __shared__ int64_t s_need;
+  __shared__ int s_cand_n;
   pdl_wait();
   const int lh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -143,15 +149,17 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
   // order.
   uint32_t prefix = 0, pmask = 0;
   int64_t need = C;
+  int64_t list_n = -1;  // after the first pass: the candidate list's length, or -1 (scan all)
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     for (int b = lane; b < 256; b += 32) whist[warp][b] = 0;
     __syncwarp();
-    for (int64_t base = int64_t(warp) * 32; base < n_c; base += kSelThreads) {
+    const int64_t n_scan = list_n < 0 ? n_c : list_n;
+    for (int64_t base = int64_t(warp) * 32; base < n_scan; base += kSelThreads) {
       const int64_t j = base + lane;
       uint32_t bin = 256;  // no bin
-      if (j < n_c) {
-        const uint32_t key = key_at(j);
+      if (j < n_scan) {
+        const uint32_t key = list_n < 0 ? key_at(j) : cand[j];
         if ((key & pmask) == prefix) bin = (key >> shift) & 255u;
       }
       const unsigned grp = __match_any_sync(0xffffffffu, bin);
@@ -198,44 +206,78 @@ select_token_kernel(int64_t n_c, int64_t S, int64_t R, int64_t N, int cached,
     prefix = s_prefix;
     need = s_need;
     pmask |= 255u << shift;
+    if (pass == 0 && cand_cap > 0) {
+      // the keys left in the running (top byte = the threshold's) as a list
+      if (tid == 0) s_cand_n = 0;
+      __syncthreads();
+      for (int64_t base = int64_t(warp) * 32; base < n_c; base += kSelThreads) {
+        const int64_t j = base + lane;
+        const uint32_t key = j < n_c ? key_at(j) : 0u;
+        const bool hit = j < n_c && (key & pmask) == prefix;
+        const unsigned bh = __ballot_sync(0xffffffffu, hit);
+        int at = 0;
+        if (lane == 0 && bh) at = atomicAdd(&s_cand_n, __popc(bh));
+        at = __shfl_sync(0xffffffffu, at, 0) + __popc(bh & ((1u << lane) - 1u));
+        if (hit && at < cand_cap) cand[at] = key;
+      }
+      __syncthreads();
+      if (s_cand_n <= cand_cap) list_n = s_cand_n;  // else every pass scans all keys
+    }
     __syncthreads();
   }
   const uint32_t t = prefix;  // exact key of the C-th largest score
   // Stable compaction in index order: every key > t, and the first `need`
   // keys == t.  Before position j, gt_before keys > t and eq_before keys == t
-  // occur, of which min(eq_before, need) are taken, so one scan of the
-  // packed pair (gt, eq) per chunk gives every destination.
-  int64_t gt_seen = 0, eq_seen = 0;
-  for (int64_t c0 = 0; c0 < n_c; c0 += kSelThreads) {
-    const int64_t j = c0 + tid;
-    const uint32_t key = j < n_c ? key_at(j) : 0u;
-    const bool gt = j < n_c && key > t;
-    const bool eq = j < n_c && key == t;
-    const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) warp_tot[warp] = int(__popc(bg) | (__popc(be) << 16));
-    __syncthreads();
-    if (warp == 0) {  // exclusive prefix of the packed (gt, eq) counts over the warps
-      const int c = warp_tot[lane];
-      int incl = c;
+  // occur, of which min(eq_before, need) are taken.  Warp w owns the
+  // contiguous keys [w0, w1): a first sweep counts its (gt, eq) keys, one
+  // block scan gives every warp its counts before w0, a second sweep writes.
+  const int64_t per_warp = ((n_c + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
+  const int64_t w0 = int64_t(warp) * per_warp;
+  const int64_t w1 = w0 + per_warp < n_c ? w0 + per_warp : n_c;
+  int gt_w = 0, eq_w = 0;
+  for (int64_t j0 = w0; j0 < w1; j0 += 32) {
+    const int64_t j = j0 + lane;
+    const uint32_t key = j < w1 ? key_at(j) : 0u;
+    gt_w += __popc(__ballot_sync(0xffffffffu, j < w1 && key > t));
+    eq_w += __popc(__ballot_sync(0xffffffffu, j < w1 && key == t));
+  }
+  if (lane == 0) {
+    warp_gt[warp] = gt_w;
+    warp_eq[warp] = eq_w;
+  }
+  __syncthreads();
+  if (warp == 0) {  // exclusive prefixes of the per-warp counts, in warp order
+    const int g = warp_gt[lane], e = warp_eq[lane];
+    int ig = g, ie = e;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vg = __shfl_up_sync(0xffffffffu, ig, o), ve = __shfl_up_sync(0xffffffffu, ie, o);
+      if (lane >= o) {
+        ig += vg;
+        ie += ve;
       }
-      warp_pre[lane] = incl - c;
-      if (lane == 31) warp_pre[32] = incl;
     }
-    __syncthreads();
-    const int before = warp_pre[warp], total = warp_pre[32];
-    const unsigned below = (1u << lane) - 1u;
-    const int64_t gt_before = gt_seen + (before & 0xFFFF) + __popc(bg & below);
-    const int64_t eq_before = eq_seen + (before >> 16) + __popc(be & below);
+    __syncwarp();
+    warp_gt[lane] = ig - g;
+    warp_eq[lane] = ie - e;
+  }
+  __syncthreads();
+  int64_t gt_seen = warp_gt[warp], eq_seen = warp_eq[warp];
+  const unsigned below = (1u << lane) - 1u;
+  for (int64_t j0 = w0; j0 < w1; j0 += 32) {
+    const int64_t j = j0 + lane;
+    const uint32_t key = j < w1 ? key_at(j) : 0u;
+    const bool gt = j < w1 && key > t;
+    const bool eq = j < w1 && key == t;
+    const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+    const int64_t gt_before = gt_seen + __popc(bg & below);
+    const int64_t eq_before = eq_seen + __popc(be & below);
     if (gt || (eq && eq_before < need)) {
       const int64_t pos = gt_before + (eq_before < need ? eq_before : need);
       out[S + pos] = int32_t(S + j);
     }
-    gt_seen += total & 0xFFFF;
-    eq_seen += total >> 16;
+    gt_seen += __popc(bg);
+    eq_seen += __popc(be);
   }
 }
 
@@ -330,14 +372,16 @@ cudaError_t launch_select_token(const Dims& d, const float* seg_score, const int
                                 int32_t* kept_idx, int32_t* kept_cnt, int32_t* status,
                                 cudaStream_t s) {
   const int cached = d.nseg <= kSelCacheKeys;
-  const size_t smem = cached ? sizeof(uint32_t) * size_t(d.nseg > 0 ? d.nseg : 1) : 0;
+  const int cand_cap = d.nseg <= kSelCandMaxKeys ? int(kSelCandKeys) : 0;
+  const size_t smem = sizeof(uint32_t) * ((cached ? size_t(d.nseg) : 0) + size_t(cand_cap) + 1);
+  static_assert(kSelCandMaxKeys + kSelCandKeys <= kSelCacheKeys, "dynamic shared memory bound");
   cudaError_t e = cudaFuncSetAttribute(select_token_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(sizeof(uint32_t) * kSelCacheKeys));
+                                       int(sizeof(uint32_t) * (kSelCacheKeys + 1)));
   if (e != cudaSuccess) return e;
   return launch_kernel(select_token_kernel, dim3(d.LH), dim3(kSelThreads), smem, s, d.pdl,
-                       d.nseg, d.S, d.R, d.N, cached, seg_score, k_per_head, kept_idx, kept_cnt,
-                       status);
+                       d.nseg, d.S, d.R, d.N, cached, cand_cap, seg_score, k_per_head, kept_idx,
+                       kept_cnt, status);
 }
 
 }  // namespace fkv

@@ -258,7 +258,8 @@ def hw_rates(dev):
     mma = {}
     for name, shape, busy in (("qk_ss_m128n128k16", 6, 0), ("pv_ts_m128n128k16", 7, 0),
                               ("ss_m128n256k16", 2, 0), ("ss_m128n64k16", 3, 0),
-                              ("qk_with_two_busy_warps", 6, 1)):
+                              ("qk_with_two_busy_warps", 6, 1),
+                              ("e4m3_qk_ss_m128n128k32", 8, 0), ("e4m3_pv_ts_m128n128k32", 9, 0)):
         for _ in range(2):
             if lib.fkv_diag_mma_rate(shape, n, busy, cyc.data_ptr(), ws.data_ptr(), s) != 0:
                 return None
@@ -717,7 +718,7 @@ def _attend_sources():
 
 def _attend_fp8_sources():
     """Source files of the e4m3 attention kernel."""
-    return ["attend_fp8_sm100.cu", "attend_common.cuh", "sm100_common.cuh"]
+    return ["attend_fp8_sm100.cu", "attend_common.cuh", "sm100_common.cuh", "f8_common.cuh"]
 
 
 # --------------------------------------------------------------------------- CPU oracle

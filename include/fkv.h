@@ -202,7 +202,9 @@ int32_t fkv_diag_attend_timeout(const fkv_params_t* p, const void* q_cur, const 
  *    (the P.V step: V stored [keys][dims]), 2 = M128 N256, 3 = M128 N64,
  *    4 = shape 0 with an MN-major B, 5 = shape 1 with a K-major B, 6 and 7
  *    = shapes 0 and 1 issued eight at a time through the attention kernel's
- *    own issue code; n_mma a multiple of 8.  busy != 0
+ *    own issue code, 8 and 9 = the e4m3 attention's M128 N128 K32
+ *    kind::f8f6f4 Q.K^T and P.V (A from tensor memory, MN-major B) issued
+ *    four at a time through its issue code; n_mma a multiple of 8.  busy != 0
  *    keeps two more warps of the issuer's sub-partition
  *    running an FMA + ex2 loop meanwhile.  cycles: device int64[4];
  *    cycles[0] = SM cycles to issue the n MMAs, cycles[1] = until they have
@@ -448,8 +450,10 @@ int32_t fkv_attend_compressed_fp8(const fkv_params_t* p, const fkv_fp8_cache_t* 
                                   const int32_t* kept_cnt, void* out, void* ws, void* stream);
 
 /* Steps 1-5 with the e4m3 cache in one call: score and select as fkv_step,
- * then fkv_compact_gather_fp8, fkv_quantize_chunk_fp8 and
- * fkv_attend_compressed_fp8, all enqueued on `stream` in that order.  io as
+ * then the work of fkv_compact_gather_fp8 and fkv_quantize_chunk_fp8 (one
+ * launch) and fkv_attend_compressed_fp8, all enqueued on `stream` in that
+ * order, each kernel after the first a programmatic dependent of the one
+ * before (as in fkv_step).  io as
  * for fkv_step (frame mode), except that io->k_comp / io->v_comp are not used
  * (may be NULL); c holds every e4m3 operand.  Same support limits as
  * fkv_attend_compressed_fp8; every host-side check runs before the first

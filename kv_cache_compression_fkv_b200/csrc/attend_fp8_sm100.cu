@@ -29,6 +29,7 @@
 
 #include "fkv_internal.cuh"
 #include "sm100_common.cuh"
+#include "f8_common.cuh"
 #include "attend_common.cuh"
 
 namespace fkv {
@@ -55,13 +56,6 @@ constexpr float kRescaleLog2 = 8.0f;
 #endif
 constexpr int kPolyEvery = FKV_F8_POLY_EVERY;
 
-// kind::f8f6f4 instruction descriptor: fp32 accumulator (bit 4), A and B
-// e4m3 (format 0 in bits 7-9 and 10-12), B MN-major flag (bit 16), N >> 3
-// (bits 17-22), M >> 4 (bits 24-28); A K-major, dense, no negation.
-__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major) {
-  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | (uint32_t(N >> 3) << 17) |
-         (uint32_t(M >> 4) << 24);
-}
 constexpr uint32_t kIdescQK = idesc_e4m3(128, 128, false);
 constexpr uint32_t kIdescPV = idesc_e4m3(128, 128, true);
 
@@ -102,91 +96,10 @@ struct Args {
   int32_t* status;
 };
 
-// D[tmem] (+)= A[smem] * B[smem]^T, both e4m3.
-__device__ __forceinline__ void mma_ss_e4m3(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem], A (e4m3, 4 per 32-bit column) from tensor memory.
-__device__ __forceinline__ void mma_ts_e4m3(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// The issuer's lookahead form of the four MMAs of a group (see mma8_ss_probe):
-// a non-blocking test of the next group's K / V barrier is issued before the
-// MMAs and read after them.  Step k: A and B 32 bytes (2 descriptor units)
-// further along the row (S), or A 8 tensor-memory columns and B 32 keys = 4 KB
-// (256 descriptor units) further (P.V).
-__device__ __forceinline__ uint32_t mma4_ss_e4m3_probe(uint32_t d, uint64_t a0, uint64_t b0,
-                                                       uint32_t idesc, uint32_t acc_first,
-                                                       uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred t, p, one;\n\t.reg .b64 a, b;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 t, [%5], %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "setp.eq.b32 one, 0, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], %2, %3, %7, p;\n\t"
-      "add.s64 a, %2, 2;\n\tadd.s64 b, %3, 2;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %7, one;\n\t"
-      "add.s64 a, %2, 4;\n\tadd.s64 b, %3, 4;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %7, one;\n\t"
-      "add.s64 a, %2, 6;\n\tadd.s64 b, %3, 6;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], a, b, %7, one;\n\t"
-      "selp.u32 %0, 1, 0, t;\n\t}\n"
-      : "=r"(ok)
-      : "r"(d), "l"(a0), "l"(b0), "r"(acc_first), "r"(smem_u32(bar)), "r"(parity), "r"(idesc)
-      : "memory");
-  return ok;
-}
-__device__ __forceinline__ uint32_t mma4_ts_e4m3_probe(uint32_t d, uint32_t a0, uint64_t b0,
-                                                       uint32_t idesc, uint32_t acc_first,
-                                                       uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred t, p, one;\n\t.reg .b32 a;\n\t.reg .b64 b;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 t, [%5], %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "setp.eq.b32 one, 0, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [%2], %3, %7, p;\n\t"
-      "add.u32 a, %2, 8;\n\tadd.s64 b, %3, 256;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %7, one;\n\t"
-      "add.u32 a, %2, 16;\n\tadd.s64 b, %3, 512;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %7, one;\n\t"
-      "add.u32 a, %2, 24;\n\tadd.s64 b, %3, 768;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%1], [a], b, %7, one;\n\t"
-      "selp.u32 %0, 1, 0, t;\n\t}\n"
-      : "=r"(ok)
-      : "r"(d), "r"(a0), "l"(b0), "r"(acc_first), "r"(smem_u32(bar)), "r"(parity), "r"(idesc)
-      : "memory");
-  return ok;
-}
 #ifndef FKV_F8_ISSUE_LOOKAHEAD
 #define FKV_F8_ISSUE_LOOKAHEAD 0
 #endif
 
-// K-major e4m3 tile: rows 128 B apart, 8-row groups 1024 B apart; step k
-// (32 elements) lives 32 B further along the row.
-__device__ __forceinline__ uint64_t kmajor8_desc(uint32_t tile_saddr, int k) {
-  return sw128_desc(tile_saddr + uint32_t(k) * 32u, 16u, 1024u);
-}
-// MN-major e4m3 V tile ([keys][dims], 128 dims = one swizzle atom wide): key
-// rows 128 B apart, 8-row groups 1024 B apart (SBO); step k = 32 keys = 4 KB.
-// With a single atom across N the leading offset has no next atom to point
-// to; it is given the minimum (16 B), which keeps any address inside the tile.
-__device__ __forceinline__ uint64_t mnmajor8_desc(uint32_t tile_saddr, int k) {
-  return sw128_desc(tile_saddr + uint32_t(k) * 4096u, 16u, 1024u);
-}
 // Four probabilities -> four e4m3 codes in one 32-bit word, the first in the low byte.
 __device__ __forceinline__ uint32_t pack_e4m3x4(float2 a, float2 b) {
   const uint32_t lo = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
@@ -234,6 +147,9 @@ attend_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // Everything above is on-chip; global memory is touched only once the
+  // kernel before this one has completed (programmatic dependent launch).
+  pdl_wait();
   if (warp >= 8) {
     regs_decrease<kControlRegs>();
   if (warp == kProducerWarp) {
@@ -621,8 +537,8 @@ cudaError_t launch_attend_fp8_sm100(const Dims& d, const fkv_fp8_cache_t& c,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem));
   if (e != cudaSuccess) return e;
   const int grid = a.n_tiles < num_sms() ? a.n_tiles : num_sms();
-  attend_fp8_kernel<<<grid, kThreads, kSmem, s>>>(tq, tkc, tvc, tkn, tvn, a);
-  return cudaGetLastError();
+  return launch_kernel(attend_fp8_kernel, dim3(grid), dim3(kThreads), kSmem, s, d.pdl, tq, tkc,
+                       tvc, tkn, tvn, a);
 }
 
 }  // namespace fkv

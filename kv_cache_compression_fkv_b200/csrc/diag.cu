@@ -5,6 +5,7 @@
 // caller data.
 #include "fkv_internal.cuh"
 #include "sm100_common.cuh"
+#include "f8_common.cuh"
 
 namespace fkv {
 namespace sm100 {
@@ -20,15 +21,31 @@ constexpr uint32_t kDiagSmem = 3 * 32768 + 1024;  // A 32 KB + B 64 KB, 1 KB ali
 //   4  as 0 with an MN-major B  5  as 1 with a K-major B
 //   6  as 0, 7  as 1, issued in groups of eight through the attention
 //      kernel's own issue helpers (mma8_ss_probe, mma8_ts_probe)
+//   8  kind::f8f6f4 (e4m3) M128 N128 K32, A and B K-major in shared memory
+//      (the e4m3 attention's Q.K^T), 9  e4m3 with A from tensor memory and
+//      an MN-major B (its P.V); both in groups of four through the e4m3
+//      kernel's issue helpers.  An e4m3 K32 MMA is as many FLOPs as two bf16
+//      K16 ones, at twice the nominal rate: 64 cycles.
 // Shapes 0-5 issue straight-line code with compile-time operand offsets, so
 // the issue loop holds nothing but the MMAs and their address arithmetic.
 template <int kShape>
 __device__ __forceinline__ void issue8(uint32_t tm, uint64_t da, uint64_t db, uint64_t dv,
-                                       uint64_t* probe_bar) {
+                                       uint64_t* probe_bar, uint32_t da_base, uint32_t db_base) {
   // operands stay inside A [0, 32 KB) and B [32 KB, 96 KB) of the shared
   // buffer; accumulators and the tensor-memory A inside the 512 columns
   constexpr uint32_t kKOff[8] = {0, 2, 4, 6, 1024, 1026, 1028, 1030};  // K-major steps
-  if constexpr (kShape == 6) {
+  if constexpr (kShape == 8) {
+    // e4m3 tiles: A [0, 16 KB), B [32 KB, 48 KB); step k = 32 B (K-major) or
+    // 4 KB (MN-major), four steps per group
+    const uint64_t a8 = f8::kmajor8_desc(uint32_t(da_base), 0), b8 = f8::kmajor8_desc(uint32_t(db_base), 0);
+    for (int g = 0; g < 2; ++g)
+      (void)f8::mma4_ss_e4m3_probe(tm, a8, b8, f8::idesc_e4m3(128, 128, false), 1u, probe_bar, 0u);
+  } else if constexpr (kShape == 9) {
+    const uint64_t v8 = f8::mnmajor8_desc(uint32_t(db_base), 0);
+    for (int g = 0; g < 2; ++g)
+      (void)f8::mma4_ts_e4m3_probe(tm + 384, tm + 256, v8, f8::idesc_e4m3(128, 128, true), 1u,
+                                   probe_bar, 0u);
+  } else if constexpr (kShape == 6) {
     (void)mma8_ss_probe(tm, da, db, idesc_bf16(128, 128, false), 1u, probe_bar, 0u);
   } else if constexpr (kShape == 7) {
     (void)mma8_ts_probe(tm + 384, tm + 256, dv, idesc_bf16(128, 128, true), 1u, probe_bar, 0u);
@@ -82,7 +99,8 @@ mma_rate_kernel(int n, int busy, long long* cycles, int32_t* status) {
       const uint64_t da = kmajor_desc(smem_u32(sm), 0), db = kmajor_desc(smem_u32(sm + 32768), 0);
       const uint64_t dv = mnmajor_desc(smem_u32(sm + 32768), 0);
       const long long t0 = clock64();
-      for (int i = 0; i < n; i += 8) issue8<kShape>(tm, da, db, dv, &probe_bar);
+      for (int i = 0; i < n; i += 8)
+        issue8<kShape>(tm, da, db, dv, &probe_bar, smem_u32(sm), smem_u32(sm + 32768));
       const long long t1 = clock64();
       mma_commit(&bar);
       const bool ok = mbar_wait(&bar, 0, &abort_flag);
@@ -136,10 +154,11 @@ __global__ void __launch_bounds__(512, 1) ex2_rate_kernel(int n, int warps, long
 cudaError_t launch_diag_mma_rate(int shape, int n, int busy, long long* cycles, int32_t* status,
                                  cudaStream_t s) {
   using namespace sm100;
-  void (*const kernels[8])(int, int, long long*, int32_t*) = {
+  void (*const kernels[10])(int, int, long long*, int32_t*) = {
       mma_rate_kernel<0>, mma_rate_kernel<1>, mma_rate_kernel<2>, mma_rate_kernel<3>,
-      mma_rate_kernel<4>, mma_rate_kernel<5>, mma_rate_kernel<6>, mma_rate_kernel<7>};
-  if (shape < 0 || shape > 7) return cudaErrorInvalidValue;
+      mma_rate_kernel<4>, mma_rate_kernel<5>, mma_rate_kernel<6>, mma_rate_kernel<7>,
+      mma_rate_kernel<8>, mma_rate_kernel<9>};
+  if (shape < 0 || shape > 9) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kernels[shape], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kDiagSmem));
   if (e != cudaSuccess) return e;

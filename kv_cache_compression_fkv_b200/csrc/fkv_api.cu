@@ -261,7 +261,7 @@ int32_t fkv_exp2_emulated(const float* x, float* y, int64_t n, void* stream) {
 
 int32_t fkv_diag_mma_rate(int32_t shape, int32_t n_mma, int32_t busy, int64_t* cycles, void* ws,
                           void* stream) {
-  if (shape < 0 || shape > 7 || n_mma < 8 || n_mma > 4096 || n_mma % 8 != 0)
+  if (shape < 0 || shape > 9 || n_mma < 8 || n_mma > 4096 || n_mma % 8 != 0)
     return FKV_ERR_SHAPE;
   if (!cycles) return FKV_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FKV_ERR_WORKSPACE;
@@ -517,10 +517,8 @@ int32_t fkv_compact_gather_fp8(const fkv_params_t* p, const void* k_hist, const 
     return FKV_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws)) != FKV_OK) return st;
   if (d.F == 0) return FKV_OK;  // nothing can be kept
-  return cuda_status(launch_quant_segments(
-      d, int(d.max_kept), d.N, d.comp_rows, kept_idx, kept_cnt, k_hist, v_hist, c->k_comp,
-      c->v_comp, c->k_comp_scale, c->v_comp_scale, status_ptr(ws),
-      static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_quant_kept(d, kept_idx, kept_cnt, k_hist, v_hist, *c, status_ptr(ws),
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 int32_t fkv_quantize_chunk_fp8(const fkv_params_t* p, const void* q_cur, const void* k_cur,
@@ -538,12 +536,8 @@ int32_t fkv_quantize_chunk_fp8(const fkv_params_t* p, const void* q_cur, const v
       !aligned4(c->k_cur_scale) || !aligned4(c->v_cur_scale))
     return FKV_ERR_INVALID_ARG;
   if ((st = check_ws(d, ws)) != FKV_OK) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if ((st = cuda_status(launch_quant_segments(d, d.Fc, d.Lq, d.Lq, nullptr, nullptr, k_cur, v_cur,
-                                              c->k_cur, c->v_cur, c->k_cur_scale,
-                                              c->v_cur_scale, status_ptr(ws), s))))
-    return st;
-  return cuda_status(launch_quant_rows(d, q_cur, c->q_cur, c->q_scale, s));
+  return cuda_status(launch_quant_chunk(d, q_cur, k_cur, v_cur, *c, status_ptr(ws),
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 // Host-side checks of the e4m3 operands that the given steps use.
@@ -609,21 +603,19 @@ int32_t fkv_step_fp8(const fkv_params_t* p, const fkv_step_io_t* io, const fkv_f
   if ((st = do_score(d, io->q_cur, io->q_score, io->k_hist, io->k_cur, io->head_role,
                      io->seg_score, ws, s)))
     return st;
-  if ((st = do_select(d, io->seg_score, io->head_role, io->static_mask, io->k_per_head,
+  // as in fkv_step: every kernel after the first is a programmatic dependent
+  Dims dp = d;
+  dp.pdl = d.F > 0;
+  if ((st = do_select(dp, io->seg_score, io->head_role, io->static_mask, io->k_per_head,
                       io->kept_idx, io->kept_cnt, ws, s)))
     return st;
-  if (d.F > 0 &&
-      (st = cuda_status(launch_quant_segments(d, int(d.max_kept), d.N, d.comp_rows, io->kept_idx,
-                                              io->kept_cnt, io->k_hist, io->v_hist, c->k_comp,
-                                              c->v_comp, c->k_comp_scale, c->v_comp_scale,
-                                              status_ptr(ws), s))))
+  dp.pdl = true;
+  // kept segments, the chunk's segments and its query rows: one launch
+  if ((st = cuda_status(launch_quant_step(dp, io->kept_idx, io->kept_cnt, io->k_hist, io->v_hist,
+                                          io->q_cur, io->k_cur, io->v_cur, *c, status_ptr(ws),
+                                          s))))
     return st;
-  if ((st = cuda_status(launch_quant_segments(d, d.Fc, d.Lq, d.Lq, nullptr, nullptr, io->k_cur,
-                                              io->v_cur, c->k_cur, c->v_cur, c->k_cur_scale,
-                                              c->v_cur_scale, status_ptr(ws), s))))
-    return st;
-  if ((st = cuda_status(launch_quant_rows(d, io->q_cur, c->q_cur, c->q_scale, s)))) return st;
-  return cuda_status(launch_attend_fp8_sm100(d, *c, io->kept_cnt, io->out, status_ptr(ws), s));
+  return cuda_status(launch_attend_fp8_sm100(dp, *c, io->kept_cnt, io->out, status_ptr(ws), s));
 }
 
 }  // extern "C"

@@ -70,6 +70,7 @@ struct WsLayout {
 
 WsLayout ws_layout(const Dims& d);
 
+
 // Programmatic dependent launch.  Inside one call sequence (fkv_step), every
 // kernel after the first is launched so that the launch is prepared while its
 // predecessor on the stream is still running and its CTAs start as soon as
@@ -184,13 +185,19 @@ cudaError_t launch_exp2_poly(const float* x, float* y, int64_t n, cudaStream_t s
 cudaError_t launch_diag_mma_rate(int shape, int n, int busy, long long* cycles, int32_t* status,
                                  cudaStream_t s);
 cudaError_t launch_diag_ex2_rate(int n, int warps, long long* cycles, cudaStream_t s);
-cudaError_t launch_quant_segments(const Dims& d, int n_slots, int64_t src_rows, int64_t dst_rows,
-                                  const int32_t* kept_idx, const int32_t* kept_cnt,
-                                  const void* src_k, const void* src_v, void* dst_k, void* dst_v,
-                                  float* scale_k, float* scale_v, int32_t* status,
-                                  cudaStream_t s);
-cudaError_t launch_quant_rows(const Dims& d, const void* src, void* dst, float* scales,
-                              cudaStream_t s);
+// e4m3 quantisation (quant_fp8.cu): the kept history segments into the
+// compressed cache, the chunk's segments and query rows, or all three in one
+// launch (the fp8 step).
+cudaError_t launch_quant_kept(const Dims& d, const int32_t* kept_idx, const int32_t* kept_cnt,
+                              const void* k_hist, const void* v_hist, const fkv_fp8_cache_t& c,
+                              int32_t* status, cudaStream_t s);
+cudaError_t launch_quant_chunk(const Dims& d, const void* q_cur, const void* k_cur,
+                               const void* v_cur, const fkv_fp8_cache_t& c, int32_t* status,
+                               cudaStream_t s);
+cudaError_t launch_quant_step(const Dims& d, const int32_t* kept_idx, const int32_t* kept_cnt,
+                              const void* k_hist, const void* v_hist, const void* q_cur,
+                              const void* k_cur, const void* v_cur, const fkv_fp8_cache_t& c,
+                              int32_t* status, cudaStream_t s);
 cudaError_t launch_attend_fp8_sm100(const Dims& d, const fkv_fp8_cache_t& c,
                                     const int32_t* kept_cnt, void* out, int32_t* status,
                                     cudaStream_t s);

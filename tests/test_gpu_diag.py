@@ -46,11 +46,12 @@ def _ex2(warps, n=4096):
 
 
 def test_mma_issue_keeps_the_tensor_pipe_busy(cuda_device):
-    r = {shape: _mma(shape) for shape in range(8)}
+    r = {shape: _mma(shape) for shape in range(10)}
     busy_issue, _ = _mma(6, busy=1)
-    names = ["QK", "PV", "N256", "N64", "SS MN-major B", "TS K-major B", "QK probe", "PV probe"]
+    names = ["QK", "PV", "N256", "N64", "SS MN-major B", "TS K-major B", "QK probe", "PV probe",
+             "e4m3 QK", "e4m3 PV"]
     print("cycles per MMA (issue/complete): " +
-          ", ".join(f"{names[k]} {r[k][0]:.1f}/{r[k][1]:.1f}" for k in range(8)) +
+          ", ".join(f"{names[k]} {r[k][0]:.1f}/{r[k][1]:.1f}" for k in range(10)) +
           f", QK probe with busy neighbours {busy_issue:.1f}")
     qk = r[0][0]
     # M128 N128 K16 bf16 = 64 cycles of tensor work: every operand source and
@@ -60,6 +61,10 @@ def test_mma_issue_keeps_the_tensor_pipe_busy(cuda_device):
     assert 1.8 <= r[2][0] / qk <= 2.2       # N = 256: twice the work, twice the time
     assert r[3][0] < 0.9 * qk               # N = 64: faster, though not half
     assert busy_issue <= 1.1 * r[6][0]      # busy warps beside the issuer cost nothing
+    # e4m3 M128 N128 K32: 64 cycles at the nominal rate (twice bf16's FLOPs per
+    # cycle); never faster than that
+    for k in (8, 9):
+        assert 60.0 <= r[k][1] <= 200.0, names[k]
 
 
 def test_one_warp_saturates_its_mufu(cuda_device):
@@ -74,7 +79,7 @@ def test_diag_rejects_bad_sizes(cuda_device):
     cyc = torch.zeros(4, dtype=torch.int64, device="cuda")
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     s = torch.cuda.current_stream().cuda_stream
-    assert lib.fkv_diag_mma_rate(8, 256, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
+    assert lib.fkv_diag_mma_rate(10, 256, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_diag_mma_rate(0, 5000, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_diag_mma_rate(0, 12, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_diag_ex2_rate(12, 1, cyc.data_ptr(), s) == _lib.FKV_ERR_SHAPE

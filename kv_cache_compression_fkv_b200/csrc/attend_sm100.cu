@@ -23,9 +23,9 @@
 //              - m) as bf16 pairs into the first 64 columns of S_h, and
 //              rescales O_h in TMEM only when m grows by more than 2^8 (lazy
 //              rescaling: P stays <= 256, exact after the final merge).
-//              Exponentials run on the MUFU unit; FKV_POLY_EVERY = n sends
-//              one pair in n to the FMA-pipe polynomial exp2_poly2 instead
-//              (measured slower at 480P: default 0).  The lead thread of
+//              Exponentials run on the MUFU unit, except one pair in
+//              FKV_POLY_EVERY (8) that goes to the FMA-pipe polynomial
+//              exp2_poly2 (fastest of 3 ... 16 at 480P).  The lead thread of
 //              each warpgroup releases the K stage of S_h(j) and the V stage
 //              of PV_h(j-1) once it sees S_h(j) complete.
 //   warp 8     TMA: lane 0 loads Q (once per unit) and the K blocks, lane 1
@@ -94,12 +94,6 @@ static_assert(kProductionWaitCycles == kWaitCycles, "one production wait limit")
 #ifndef FKV_POLY_EVERY
 #define FKV_POLY_EVERY 8
 #endif
-// 1: each stream's logit tile is double-buffered as two 64-key halves, so the
-// next half's Q.K^T runs while the softmax works on the current one.
-#ifndef FKV_ATTN_SPLIT_S
-#define FKV_ATTN_SPLIT_S 0
-#endif
-constexpr uint32_t kIdescQK64 = idesc_bf16(128, 64, false);
 
 __host__ __device__ constexpr uint32_t col_s(int h) { return 128u * uint32_t(h); }
 __host__ __device__ constexpr uint32_t col_o(int h) { return 256u + 128u * uint32_t(h); }
@@ -113,12 +107,7 @@ struct AttnBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-#if FKV_ATTN_SPLIT_S
-  uint64_t s_full[2][2], p_full[2][2];  // per stream and 64-key half
-  uint64_t pv_last[2];                  // per stream: its last half-a PV of the unit done
-#else
   uint64_t s_full[2], p_full[2];  // per stream
-#endif
   uint64_t o_ready, o_free;       // per unit: both PV chains done / both O read
   uint64_t mma_done;
   uint64_t x_full, x_read;        // merge exchange handshake (256 arrivals each)
@@ -172,16 +161,8 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(&bars->v_empty[s], 1);
     }
     for (int h = 0; h < 2; ++h) {
-#if FKV_ATTN_SPLIT_S
-      for (int x = 0; x < 2; ++x) {
-        mbar_init(&bars->s_full[h][x], 1);
-        mbar_init(&bars->p_full[h][x], 128);
-      }
-      mbar_init(&bars->pv_last[h], 1);
-#else
       mbar_init(&bars->s_full[h], 1);
       mbar_init(&bars->p_full[h], 128);
-#endif
     }
     mbar_init(&bars->o_ready, 1);
     mbar_init(&bars->o_free, kSoftmaxThreads);
@@ -269,95 +250,6 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     // order), descriptors are precomputed, one commit per S group (the
     // softmax releases the K and V stages), and a tcgen05 fence only where
     // another thread wrote TMEM (P, and O after the epilogue).
-#if FKV_ATTN_SPLIT_S
-    // Per stream h and 64-key half x of block j: PV_hx(j-1) (4 MMAs, K = 64,
-    // P from the half's first 32 TMEM columns, V rows 64x.. of the block),
-    // then S_hx(j) = Q K[rows 64x..]^T (8 MMAs, N = 64) and its commit.
-    // Order per j: half a of both streams, then half b, so that S_hx(j) is
-    // issued as soon as the softmax has stored P_hx(j-1) and runs while the
-    // softmax works on the stream's other half.
-    if (lane == 0) {
-      uint32_t uc = 0, base = 0;
-      uint32_t pb0 = 0, pb1 = 0;  // blocks of stream 0 / 1 in earlier units (P completions)
-      bool ok = true;
-      bool withhold = a.withhold_s0 != 0 && blockIdx.x == 0;
-      const uint64_t dq = kmajor_desc(smem_u32(sm + kOffQ), 0);
-      const uint64_t dk0 = kmajor_desc(smem_u32(sm + kOffK), 0);
-      const uint64_t dv0 = mnmajor_desc(smem_u32(sm + kOffV), 0);
-      constexpr uint32_t kStageDesc = kTileBytes >> 4;  // descriptor step between ring stages
-      constexpr uint32_t kHalfDesc = (64 * 128) >> 4;   // 64 rows of 128 B into a region
-      for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++uc) {
-        const Unit t = decode(a, tile);
-        bool o_free_seen = false;
-        auto issue_pv = [&](int h, int x, int j, bool first) -> bool {
-          if (!o_free_seen) {
-            if (!mbar_wait(&bars->o_free, (uc & 1) ^ 1, abort, a.wait_cycles)) return false;
-            o_free_seen = true;
-          }
-          const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
-          const uint32_t vs = pos % kVStages, vph = (pos / kVStages) & 1;
-          if (!mbar_wait(&bars->v_full[vs], vph, abort, a.wait_cycles)) return false;
-          // P_hx(j) is completion number (blocks of stream h before this unit) + j
-          const uint32_t pn = (h ? pb1 : pb0) + uint32_t(j);
-          if (!mbar_wait(&bars->p_full[h][x], pn & 1, abort, a.wait_cycles)) return false;
-          tc_fence_after();
-          const uint64_t dv = dv0 + uint64_t(vs * kStageDesc + uint32_t(x) * kHalfDesc);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_ts(tmem + col_o(h), tmem + col_s(h) + 64u * uint32_t(x) + 8u * uint32_t(k),
-                   dv + uint64_t(k) * 128u, kIdescPV, (first && k == 0) ? 0u : 1u);
-          return true;
-        };
-        auto issue_s = [&](int h, int x, int j) -> bool {
-          const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
-          const uint32_t ks = pos % kKStages, kph = (pos / kKStages) & 1;
-          if (!mbar_wait(&bars->k_full[ks], kph, abort, a.wait_cycles)) return false;
-          const uint64_t dk = dk0 + uint64_t(ks * kStageDesc + uint32_t(x) * kHalfDesc);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            const uint64_t off = uint64_t((k >> 2) * (kRegionBytes >> 4) + (k & 3) * 2);
-            mma_ss(tmem + col_s(h) + 64u * uint32_t(x), dq + off, dk + off, kIdescQK64,
-                   k > 0 ? 1u : 0u);
-          }
-          if (withhold && h == 0 && x == 0) withhold = false;
-          else mma_commit(&bars->s_full[h][x]);
-          return true;
-        };
-        if (!(ok = mbar_wait(&bars->q_full, uc & 1, abort, a.wait_cycles))) break;
-        for (int j = 0; ok && j < t.nb0; ++j) {
-          for (int x = 0; ok && x < 2; ++x) {
-            for (int h = 0; h < 2; ++h) {
-              const int nbh = h ? t.nb1 : t.nb0;
-              if (j < nbh) {
-                if (j > 0 && !(ok = issue_pv(h, x, j - 1, j == 1 && x == 0))) break;
-                if (!(ok = issue_s(h, x, j))) break;
-              } else if (j == nbh && j > 0) {  // stream 1's last PVs, in load order
-                if (!(ok = issue_pv(h, x, j - 1, j == 1 && x == 0))) break;
-                if (x == 0) mma_commit(&bars->pv_last[h]);
-              }
-            }
-          }
-        }
-        if (!ok) break;
-        mma_commit(&bars->q_empty);  // every S of this unit issued
-        for (int h = 0; ok && h < 2; ++h) {
-          const int nbh = h ? t.nb1 : t.nb0;
-          if (nbh == 0 || (h == 1 && t.nb1 < t.nb0)) continue;
-          if (!(ok = issue_pv(h, 0, nbh - 1, nbh == 1))) break;
-          mma_commit(&bars->pv_last[h]);
-          if (!(ok = issue_pv(h, 1, nbh - 1, false))) break;
-        }
-        if (!ok) break;
-        mma_commit(&bars->o_ready);
-        base += uint32_t(t.nb);
-        pb0 += uint32_t(t.nb0);
-        pb1 += uint32_t(t.nb1);
-      }
-      // Every MMA issued here completes before TMEM is released.
-      mma_commit(&bars->mma_done);
-      drain_wait(&bars->mma_done, 0);
-    }
-#else
     if (lane == 0) {
       uint32_t uc = 0, ks = 0, kph = 0, vs = 0, vph = 0;
       uint32_t p_use[2] = {0, 0};
@@ -470,7 +362,6 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
       mma_commit(&bars->mma_done);
       drain_wait(&bars->mma_done, 0);
     }
-#endif
   }
   } else {
     regs_increase<kSoftmaxRegs>();
@@ -480,129 +371,11 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + lane_addr + col_s(h);
     uint32_t use = 0, base = 0, uc = 0;
-#if FKV_ATTN_SPLIT_S
-    uint32_t pl_use = 0;  // completions of pv_last[h] seen so far (units with blocks)
-#endif
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < a.n_tiles; tile += gridDim.x, ++uc) {
       const Unit t = decode(a, tile);
       const int mine = h ? t.nb1 : t.nb0;
       float m = -INFINITY, l = 0.f;
-#if FKV_ATTN_SPLIT_S
-      // use = blocks of this stream completed before this unit; block j's
-      // halves are completion number use + j of s_full[h][0] and [1].
-      for (int j = 0; ok && j < mine; ++j) {
-        const int b = block_of(t, h, j);
-        const bool inA = b < t.nbA;
-        const int64_t rows_left = (inA ? t.nA : a.Lq) - int64_t(inA ? b : b - t.nbA) * 128;
-        const int nv = rows_left < 128 ? int(rows_left) : 128;  // valid keys of the block
-        const uint32_t n = use + uint32_t(j);
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const int nvx = nv - 64 * x;  // valid keys of this half (may be <= 0)
-          if (!(ok = warp_wait(&bars->s_full[h][x], n & 1, abort, a.wait_cycles))) break;
-          tc_fence_after();
-          if (row == 0 && x == 1) {
-            // S_hb(j) is complete, and with it every MMA issued before it: the
-            // K stage of block j and the V stage of this stream's block j-1
-            // (its PV_hb was issued right before S_hb(j)) are free.
-            mbar_arrive(&bars->k_empty[(base + uint32_t(seq_pos(t, h, j))) % kKStages]);
-            if (j > 0) mbar_arrive(&bars->v_empty[(base + uint32_t(seq_pos(t, h, j - 1))) % kVStages]);
-          }
-          uint32_t sr[64];  // raw fp32 logits of this row's half block
-#define SV(i) __uint_as_float(sr[i])
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            tmem_ld32(tS + 64 * x + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-          tmem_ld_wait();
-          if (nvx < 64) {  // ragged: columns past the valid keys never count
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (i >= nvx) sr[i] = 0xff800000u;  // -inf
-          }
-          float mx[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = fmaxf(SV(k), SV(k + 8));
-#pragma unroll
-          for (int i = 16; i < 64; i += 16)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx[k] = fmax3(mx[k], SV(i + k), SV(i + k + 8));
-          const float bmax = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]),
-                                   fmaxf(mx[6], mx[7]));
-          const float m_new = fmaxf(m, bmax * a.sl2);  // scale > 0
-          if (j == 0 && x == 0) {
-            m = m_new;
-          } else if (__any_sync(0xffffffffu, m_new > m + kRescaleLog2)) {
-            // Every PV issued into O_h must be complete before O_h is
-            // rescaled.  The one of this stream's other half is covered by
-            // the commit of the S group issued after it: S_hb(j) for half a
-            // of block j, S_ha(j+1) (or, after the last block, pv_last[h])
-            // for half b.  Both are already issued: their P is stored.
-            bool done;
-            if (x == 0) done = warp_wait(&bars->s_full[h][1], n & 1, abort, a.wait_cycles);
-            else if (j + 1 < mine) done = warp_wait(&bars->s_full[h][0], (n + 1) & 1, abort, a.wait_cycles);
-            else done = warp_wait(&bars->pv_last[h], pl_use & 1, abort, a.wait_cycles);
-            if (!(ok = done)) break;
-            tc_fence_after();
-            const float alpha = ex2(m - m_new);
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-              uint32_t o[16];
-              tmem_ld16(tmem + lane_addr + col_o(h) + c * 16, o);
-              tmem_ld_wait();
-#pragma unroll
-              for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st16(tmem + lane_addr + col_o(h) + c * 16, o);
-            }
-            tmem_st_wait();
-            l *= alpha;
-            m = m_new;
-          }
-          float2 acc[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[k] = make_float2(0.f, 0.f);
-          const float2 sl2x2 = make_float2(a.sl2, a.sl2), negm2 = make_float2(-m, -m);
-          uint32_t pk[32];  // P of the half (bf16 pairs) over its first 32 TMEM columns
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float2 e = ffma2(make_float2(SV(2 * i), SV(2 * i + 1)), sl2x2, negm2);
-            const float2 p = (FKV_POLY_EVERY > 0 && i % (FKV_POLY_EVERY > 0 ? FKV_POLY_EVERY : 1) ==
-                                                       (FKV_POLY_EVERY > 0 ? FKV_POLY_EVERY : 1) - 1)
-                                 ? exp2_poly2(e)
-                                 : make_float2(ex2(e.x), ex2(e.y));
-            acc[i & 3] = fadd2(acc[i & 3], p);
-            pk[i] = pack_bf16(p.x, p.y);
-          }
-          tmem_st32(tS + 64 * x, pk);
-#undef SV
-          const float2 s2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
-          l += s2.x + s2.y;
-          tmem_st_wait();
-          if (x == 0 && nv < 128) {
-            // V rows past the valid keys may hold anything (P is 0 there, but
-            // 0 * NaN is not 0): zero them, for both halves, before PV_ha reads the stage.
-            const uint32_t pos = base + uint32_t(seq_pos(t, h, j));
-            const uint32_t s = pos % kVStages, u = pos / kVStages;
-            if (!(ok = warp_wait(&bars->v_full[s], u & 1, abort, a.wait_cycles))) break;
-            if (row >= nv) {
-              uint4* v0 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + row * 128);
-              uint4* v1 = reinterpret_cast<uint4*>(sm + kOffV + s * kTileBytes + kRegionBytes + row * 128);
-              const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                v0[c] = z;
-                v1[c] = z;
-              }
-            }
-            fence_proxy_async_smem();
-          }
-          tc_fence_before();
-          mbar_arrive(&bars->p_full[h][x]);
-        }
-      }
-      use += uint32_t(mine);
-      if (mine > 0) ++pl_use;
-#else
       for (int j = 0; j < mine; ++j, ++use) {
         const int b = block_of(t, h, j);
         const bool inA = b < t.nbA;
@@ -702,7 +475,6 @@ attend_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_before();
         mbar_arrive(&bars->p_full[h]);
       }
-#endif
       if (!ok) break;
       // V stage of this stream's last PV (released once both PV chains are done)
       const uint32_t last_v = mine > 0 ? (base + uint32_t(seq_pos(t, h, mine - 1))) % kVStages : 0u;

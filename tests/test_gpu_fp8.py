@@ -173,8 +173,11 @@ def test_step_fp8_equals_the_separate_calls(cuda_device):
         assert torch.equal(c[k], c2[k]), k
     cnt = o["kept_cnt"].cpu()
     for h in range(w.H):
-        rows = int(cnt[0, h]) * w.T
-        assert torch.equal(c["k_comp"][0, h, :rows], c2["k_comp"][0, h, :rows])
+        rows, n = int(cnt[0, h]) * w.T, int(cnt[0, h])
+        for k in ("k_comp", "v_comp"):
+            assert torch.equal(c[k][0, h, :rows], c2[k][0, h, :rows]), (k, h)
+        for k in ("k_comp_scale", "v_comp_scale"):
+            assert torch.equal(c[k][0, h, :n], c2[k][0, h, :n]), (k, h)
 
 
 def test_attend_fp8_1080p_sampled_rows(cuda_device):

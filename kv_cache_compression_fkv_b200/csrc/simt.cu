@@ -110,19 +110,32 @@ score_frame_partial_kernel(int D, int T_, int F, int64_t Lq, int stride, int64_t
 // frame entries per head, split consecutive pieces per frame, then `chunk`
 // entries of the chunk's own keys when they join the normaliser; G = F*split +
 // chunk entries in the row normaliser):
-//   row merge   M_i = max_g m_{g,i},  L_i = sum_g l_{g,i} 2^(m_{g,i} - M_i)
+//   frame part  (m_f, l_f) = the merge of frame f's `split` entries
+//               (m_f = max m, l_f = sum l 2^(m - m_f)); the chunk's entries
+//               form one more part;
+//   row merge   M_i = max_f m_f,  L_i = sum_f l_f 2^(m_f - M_i)
 //               (stored as (M_i, 1/L_i) in row_ml),
-//   frame mass  mass_f = sum_i c_{f,i},  c_{f,i} = sum_{g in f} l_{g,i} 2^(m_{g,i} - M_i) / L_i.
+//   frame mass  mass_f = sum_i c_{f,i},  c_{f,i} = l_f 2^(m_f - M_i) / L_i.
 // Two kernels, every sum in a fixed order (deterministic, equal frames give
 // bit-equal masses):
-//   score_rows_kernel    one warp per (head, row): lanes stride the row's
-//                        entries (contiguous), a fixed shuffle tree; c_{f,i}
-//                        is written back over the m of the frame's first
-//                        entry of the same row (each warp touches only its
-//                        own row);
+//   score_rows_kernel    one warp per (head, row): lane t merges parts t,
+//                        t + 32, ... (each read once, its entries loaded
+//                        together), writes (m_f, l_f) over the part's first
+//                        entry, the lanes' merges combine in a fixed shuffle
+//                        tree, then each lane turns its parts into c_{f,i},
+//                        written over the m of the frame's first entry (each
+//                        warp touches only its own row);
 //   score_frames_kernel  one CTA per (head, frame): threads stride the rows,
 //                        a fixed shuffle tree and a fixed warp order.
 constexpr int kRowWarps = 8;
+
+// (m, l) of the union of two partial softmax sums; empty parts are (-inf, 0).
+__device__ __forceinline__ float2 merge_part(float2 a, float2 b) {
+  const float M = fmaxf(a.x, b.x);
+  if (M == -INFINITY) return make_float2(-INFINITY, 0.f);
+  return make_float2(M, (a.y != 0.f ? a.y * exp2f(a.x - M) : 0.f) +
+                            (b.y != 0.f ? b.y * exp2f(b.x - M) : 0.f));
+}
 
 __global__ void __launch_bounds__(kRowWarps * 32)
 score_rows_kernel(int F, int split, int chunk, int E, int64_t n_s,
@@ -133,46 +146,39 @@ score_rows_kernel(int F, int split, int chunk, int E, int64_t n_s,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t i = int64_t(blockIdx.x) * kRowWarps + warp;
   if (!head_role[lh] || i >= n_s) return;  // warp-uniform
-  const int G = F * split + chunk;  // entries of the row normaliser
   float2* p = part_ml + (int64_t(lh) * n_s + i) * E;  // the row's E entries, contiguous
-  // the entry loops are unrolled so that several loads are in flight per lane
-  float M = -INFINITY;
-#pragma unroll 4
-  for (int g = lane; g < G; g += 32) M = fmaxf(M, p[g].x);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float Ls = 0.f;
-#pragma unroll 4
-  for (int g = lane; g < G; g += 32) {
-    const float2 ml = p[g];
-    if (ml.y != 0.f) Ls += ml.y * exp2f(ml.x - M);
+  const int nparts = F + (chunk > 0 ? 1 : 0);
+  // 1. each lane's parts, merged in part order
+  float2 mine = make_float2(-INFINITY, 0.f);
+  for (int f = lane; f < nparts; f += 32) {
+    const int n = f < F ? split : chunk;
+    const float2* e = p + f * split;  // the chunk part starts at F * split
+    float2 part = make_float2(-INFINITY, 0.f);
+    int g = 0;
+    for (; g + 4 <= n; g += 4) {  // four loads in flight
+      const float2 e0 = e[g], e1 = e[g + 1], e2 = e[g + 2], e3 = e[g + 3];
+      part = merge_part(part, e0);
+      part = merge_part(part, e1);
+      part = merge_part(part, e2);
+      part = merge_part(part, e3);
+    }
+    for (; g < n; ++g) part = merge_part(part, e[g]);
+    if (f < F) p[f * split] = part;  // only this lane reads it back
+    mine = merge_part(mine, part);
   }
+  // 2. the row's (M, L): a fixed shuffle tree over the lanes
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-  const float inv = 1.f / Ls;
+  for (int o = 16; o > 0; o >>= 1) {
+    const float2 other = make_float2(__shfl_xor_sync(0xffffffffu, mine.x, o),
+                                     __shfl_xor_sync(0xffffffffu, mine.y, o));
+    mine = (lane & o) ? merge_part(other, mine) : merge_part(mine, other);
+  }
+  const float M = mine.x, inv = 1.f / mine.y;
   if (lane == 0) row_ml[int64_t(lh) * n_s + i] = make_float2(M, inv);
-  float c[4];  // frames lane, lane + 32, ... (up to 128 frames per pass)
-  for (int f0 = 0; f0 < F; f0 += 128) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int f = f0 + lane + 32 * u;
-      c[u] = 0.f;
-      if (f < F) {
-        float t = 0.f;
-#pragma unroll 4
-        for (int s2 = 0; s2 < split; ++s2) {
-          const float2 ml = p[f * split + s2];
-          if (ml.y != 0.f) t += ml.y * exp2f(ml.x - M);
-        }
-        c[u] = t * inv;
-      }
-    }
-    __syncwarp();  // every lane has read the entries this pass overwrites
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int f = f0 + lane + 32 * u;
-      if (f < F) p[f * split].x = c[u];
-    }
+  // 3. c_{f,i} over the m of each frame's first entry
+  for (int f = lane; f < F; f += 32) {
+    const float2 part = p[f * split];
+    p[f * split].x = part.y != 0.f ? part.y * exp2f(part.x - M) * inv : 0.f;
   }
 }
 

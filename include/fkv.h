@@ -195,21 +195,20 @@ int32_t fkv_diag_attend_timeout(const fkv_params_t* p, const void* q_cur, const 
 
 /* Diagnostics of the hardware rates the attention kernel's design rests on
  * (one CTA per SM; CTA 0 reports; no caller data is touched):
- *  - fkv_diag_mma_rate: one thread issues n_mma (8..4096) tcgen05.mma
- *    back to back into one accumulator, bf16 operands, fp32 accumulation;
- *    shape 0 = M128 N128 K16 from shared memory, B K-major (the Q.K^T
- *    step), 1 = M128 N128 K16 with A from tensor memory and an MN-major B
- *    (the P.V step: V stored [keys][dims]), 2 = M128 N256, 3 = M128 N64,
- *    4 = shape 0 with an MN-major B, 5 = shape 1 with a K-major B, 6 and 7
- *    = shapes 0 and 1 issued eight at a time through the attention kernel's
- *    own issue code, 8 and 9 = the e4m3 attention's M128 N128 K32
- *    kind::f8f6f4 Q.K^T and P.V (A from tensor memory, MN-major B) issued
- *    four at a time through its issue code; n_mma a multiple of 8.  busy != 0
- *    keeps two more warps of the issuer's sub-partition
- *    running an FMA + ex2 loop meanwhile.  cycles: device int64[4];
- *    cycles[0] = SM cycles to issue the n MMAs, cycles[1] = until they have
- *    completed.  ws: a workspace (>= 256 B, 256-B aligned) whose status word
- *    records FKV_ERR_TIMEOUT if the completion wait gave up.
+ *  - fkv_diag_mma_rate: one thread issues n_mma (8..4096, a multiple of 8)
+ *    tcgen05.mma back to back into one fp32 accumulator in tensor memory.
+ *    Shapes (bf16 unless noted): 0 = M128 N128 K16, A and B K-major in
+ *    shared memory (the Q.K^T step); 1 = M128 N128 K16, A from tensor memory,
+ *    B MN-major (the P.V step: V stored [keys][dims]); 2 = M128 N256; 3 =
+ *    M128 N64; 4 = shape 0 with an MN-major B; 5 = shape 1 with a K-major B;
+ *    6, 7 = shapes 0, 1 issued eight at a time through the attention
+ *    kernel's own issue code; 8, 9 = the e4m3 attention's M128 N128 K32
+ *    kind::f8f6f4 Q.K^T and P.V, four at a time through its issue code.
+ *    busy != 0 keeps two more warps of the issuer's sub-partition running an
+ *    FMA + ex2 loop meanwhile.  cycles: device int64[4]; cycles[0] = SM
+ *    cycles to issue the n MMAs, cycles[1] = until they have completed.  ws:
+ *    a workspace (>= 256 B, 256-B aligned) whose status word records
+ *    FKV_ERR_TIMEOUT if the completion wait gave up.
  *  - fkv_diag_ex2_rate: `warps` (1..4) warps per SM sub-partition each run
  *    n (multiple of 8, <= 2^20) ex2.approx.ftz.f32 in 8 independent chains;
  *    cycles: device int64[2]; cycles[0] = SM cycles of one warp.

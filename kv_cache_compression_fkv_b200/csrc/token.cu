@@ -40,7 +40,10 @@ qsum_kernel(int D, int64_t n_q, const T* __restrict__ q_score, float* __restrict
 // 16-byte load per row; 64 row groups (r = g mod 64) summed in order, then
 // the 64 group sums per dim added in a fixed order.
 constexpr int kQsumRowGroups = 64;
-constexpr int kQsumBatch = 8;
+#ifndef FKV_QSUM_BATCH
+#define FKV_QSUM_BATCH 8
+#endif
+constexpr int kQsumBatch = FKV_QSUM_BATCH;
 __global__ void __launch_bounds__(1024)
 qsum_bf16_kernel(int64_t n_q, const uint4* __restrict__ q_score, float* __restrict__ qbar) {
   __shared__ float part[kQsumRowGroups][128];
@@ -81,7 +84,13 @@ qsum_bf16_kernel(int64_t n_q, const uint4* __restrict__ q_score, float* __restri
 
 // bf16, D = 128.  grid = (blocks per head, L*H), 256 threads.
 constexpr int kPhiThreads = 256;
-constexpr int kPhiUnroll = 4;  // row pairs in flight per warp
+#ifndef FKV_PHI_CTAS_PER_SM
+#define FKV_PHI_CTAS_PER_SM 8
+#endif
+#ifndef FKV_PHI_UNROLL
+#define FKV_PHI_UNROLL 4
+#endif
+constexpr int kPhiUnroll = FKV_PHI_UNROLL;  // row pairs in flight per warp
 
 __global__ void __launch_bounds__(kPhiThreads)
 phi_bf16_kernel(int64_t N, int64_t S, int64_t n_c, const uint4* __restrict__ k_hist,
@@ -160,8 +169,8 @@ cudaError_t launch_score_token(const Dims& d, const void* q_score, const void* k
     qsum_kernel<float><<<d.LH, kQsumThreads, 0, s>>>(d.D, d.n_score_q,
                                                      static_cast<const float*>(q_score), qbar);
   if (d.bf16) {
-    // About 8 CTAs of 256 threads per SM over all heads.
-    int64_t per_head = (int64_t(num_sms()) * 8 + d.LH - 1) / d.LH;
+    // About FKV_PHI_CTAS_PER_SM CTAs of 256 threads per SM over all heads.
+    int64_t per_head = (int64_t(num_sms()) * FKV_PHI_CTAS_PER_SM + d.LH - 1) / d.LH;
     const int64_t rows_per_block = (kPhiThreads / 32) * 2 * kPhiUnroll;
     const int64_t need = (d.nseg + rows_per_block - 1) / rows_per_block;
     if (per_head > need) per_head = need;

@@ -203,7 +203,8 @@ int32_t fkv_diag_attend_timeout(const fkv_params_t* p, const void* q_cur, const 
  *    M128 N64; 4 = shape 0 with an MN-major B; 5 = shape 1 with a K-major B;
  *    6, 7 = shapes 0, 1 issued eight at a time through the attention
  *    kernel's own issue code; 8, 9 = the e4m3 attention's M128 N128 K32
- *    kind::f8f6f4 Q.K^T and P.V, four at a time through its issue code.
+ *    kind::f8f6f4 Q.K^T and P.V, four at a time through its issue code;
+ *    10 = shape 0 with M = 64.
  *    busy != 0 keeps two more warps of the issuer's sub-partition running an
  *    FMA + ex2 loop meanwhile.  cycles: device int64[4]; cycles[0] = SM
  *    cycles to issue the n MMAs, cycles[1] = until they have completed.  ws:

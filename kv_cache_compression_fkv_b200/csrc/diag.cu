@@ -26,6 +26,7 @@ constexpr uint32_t kDiagSmem = 3 * 32768 + 1024;  // A 32 KB + B 64 KB, 1 KB ali
 //      an MN-major B (its P.V); both in groups of four through the e4m3
 //      kernel's issue helpers.  An e4m3 K32 MMA is as many FLOPs as two bf16
 //      K16 ones, at twice the nominal rate: 64 cycles.
+//   10 as 0 with M = 64 (a 64-row query tile: half the rows of shape 0)
 // Shapes 0-5 issue straight-line code with compile-time operand offsets, so
 // the issue loop holds nothing but the MMAs and their address arithmetic.
 template <int kShape>
@@ -55,6 +56,8 @@ __device__ __forceinline__ void issue8(uint32_t tm, uint64_t da, uint64_t db, ui
       if constexpr (kShape == 0 || kShape == 2 || kShape == 3)
         mma_ss(tm, da + kKOff[k], db + kKOff[k],
                idesc_bf16(128, kShape == 2 ? 256 : kShape == 3 ? 64 : 128, false), 1u);
+      else if constexpr (kShape == 10)
+        mma_ss(tm, da + kKOff[k], db + kKOff[k], idesc_bf16(64, 128, false), 1u);
       else if constexpr (kShape == 1)
         mma_ts(tm + 384, tm + 256 + 8 * k, dv + 128u * k, idesc_bf16(128, 128, true), 1u);
       else if constexpr (kShape == 4)
@@ -154,11 +157,11 @@ __global__ void __launch_bounds__(512, 1) ex2_rate_kernel(int n, int warps, long
 cudaError_t launch_diag_mma_rate(int shape, int n, int busy, long long* cycles, int32_t* status,
                                  cudaStream_t s) {
   using namespace sm100;
-  void (*const kernels[10])(int, int, long long*, int32_t*) = {
+  void (*const kernels[11])(int, int, long long*, int32_t*) = {
       mma_rate_kernel<0>, mma_rate_kernel<1>, mma_rate_kernel<2>, mma_rate_kernel<3>,
       mma_rate_kernel<4>, mma_rate_kernel<5>, mma_rate_kernel<6>, mma_rate_kernel<7>,
-      mma_rate_kernel<8>, mma_rate_kernel<9>};
-  if (shape < 0 || shape > 9) return cudaErrorInvalidValue;
+      mma_rate_kernel<8>, mma_rate_kernel<9>, mma_rate_kernel<10>};
+  if (shape < 0 || shape > 10) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(kernels[shape], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(kDiagSmem));
   if (e != cudaSuccess) return e;

@@ -261,7 +261,7 @@ int32_t fkv_exp2_emulated(const float* x, float* y, int64_t n, void* stream) {
 
 int32_t fkv_diag_mma_rate(int32_t shape, int32_t n_mma, int32_t busy, int64_t* cycles, void* ws,
                           void* stream) {
-  if (shape < 0 || shape > 9 || n_mma < 8 || n_mma > 4096 || n_mma % 8 != 0)
+  if (shape < 0 || shape > 10 || n_mma < 8 || n_mma > 4096 || n_mma % 8 != 0)
     return FKV_ERR_SHAPE;
   if (!cycles) return FKV_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FKV_ERR_WORKSPACE;

@@ -7,6 +7,7 @@ library's diagnostics (one CTA per SM, clock64 in CTA 0):
     layout and either A source, and through the attention's grouped issue
     helpers: the issue is not what bounds the kernel;  an N = 256 MMA takes
     twice as long, an N = 64 one is bound by the issue itself;
+  * an M = 64 MMA takes as long as an M = 128 one (half the FLOP rate);
   * one warp keeps its sub-partition's MUFU busy (about 8 cycles per ex2 warp
     instruction); two warps share it (about twice as long each).
 
@@ -46,12 +47,12 @@ def _ex2(warps, n=4096):
 
 
 def test_mma_issue_keeps_the_tensor_pipe_busy(cuda_device):
-    r = {shape: _mma(shape) for shape in range(10)}
+    r = {shape: _mma(shape) for shape in range(11)}
     busy_issue, _ = _mma(6, busy=1)
     names = ["QK", "PV", "N256", "N64", "SS MN-major B", "TS K-major B", "QK probe", "PV probe",
-             "e4m3 QK", "e4m3 PV"]
+             "e4m3 QK", "e4m3 PV", "M64"]
     print("cycles per MMA (issue/complete): " +
-          ", ".join(f"{names[k]} {r[k][0]:.1f}/{r[k][1]:.1f}" for k in range(10)) +
+          ", ".join(f"{names[k]} {r[k][0]:.1f}/{r[k][1]:.1f}" for k in range(11)) +
           f", QK probe with busy neighbours {busy_issue:.1f}")
     qk = r[0][0]
     # M128 N128 K16 bf16 = 64 cycles of tensor work: every operand source and
@@ -65,6 +66,9 @@ def test_mma_issue_keeps_the_tensor_pipe_busy(cuda_device):
     # cycle); never faster than that
     for k in (8, 9):
         assert 60.0 <= r[k][1] <= 200.0, names[k]
+    # M = 64: half the work of shape 0 in the same time (half the FLOP rate),
+    # so a 64-row tile saves no tensor time over a padded 128-row one
+    assert 0.9 * r[0][1] <= r[10][1] <= 1.1 * r[0][1]
 
 
 def test_one_warp_saturates_its_mufu(cuda_device):
@@ -79,7 +83,7 @@ def test_diag_rejects_bad_sizes(cuda_device):
     cyc = torch.zeros(4, dtype=torch.int64, device="cuda")
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
     s = torch.cuda.current_stream().cuda_stream
-    assert lib.fkv_diag_mma_rate(10, 256, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
+    assert lib.fkv_diag_mma_rate(11, 256, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_diag_mma_rate(0, 5000, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_diag_mma_rate(0, 12, 0, cyc.data_ptr(), ws.data_ptr(), s) == _lib.FKV_ERR_SHAPE
     assert lib.fkv_diag_ex2_rate(12, 1, cyc.data_ptr(), s) == _lib.FKV_ERR_SHAPE
